@@ -1,0 +1,148 @@
+"""Plant plausible mistakes in the oracle and check that some pin catches each one.
+
+Every mutation below is a slip a restatement of the method could make (a dropped term, a wrong
+sign, scale or index, a transposed grouping, a wrong tie-break). The pins of oracle_checks.py
+must not all pass on any of them. CPU only; the oracle is patched in this process only.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle.compkv as O
+import oracle_checks as C
+
+_orig = {name: getattr(O, name) for name in (
+    "block_summaries", "logit_variance_estimate", "second_order_log_mass", "head_scores",
+    "compensated_attention", "select_blocks", "block_mean_logits", "dense_attention",
+    "group_scores", "token_logits", "block_residuals", "log_partitions")}
+
+
+def _summaries_sample_var(k, v, block_size=16, n_groups=4):
+    s = _orig["block_summaries"](k, v, block_size, n_groups)
+    n = s.count.astype(float)[:, None]
+    s.var_g = s.var_g * n / np.maximum(n - 1, 1)
+    return s
+
+
+def _summaries_interleaved(k, v, block_size=16, n_groups=4):
+    k64 = np.asarray(C.np.asarray(k, dtype=float))
+    s = _orig["block_summaries"](k, v, block_size, n_groups)
+    T, d = k64.shape
+    for j in range(s.count.shape[0]):
+        kb = k64[j * block_size:(j + 1) * block_size]
+        var = kb.var(axis=0)
+        s.var_g[j] = var.reshape(d // n_groups, n_groups).mean(axis=0)
+    return s
+
+
+def _vhat_one_scale(q, summ, scale):
+    return _orig["logit_variance_estimate"](q, summ, scale) / scale
+
+
+def _logm_no_second_order(q, summ, scale):
+    return np.log(summ.count.astype(float)) + O.block_mean_logits(q, summ, scale)
+
+
+def _logm_no_count(q, summ, scale):
+    return _orig["second_order_log_mass"](q, summ, scale) - np.log(summ.count.astype(float))
+
+
+def _scores_unnormalised(q, summ, scale, mode="compkv"):
+    log_m = O.second_order_log_mass(q, summ, scale)
+    m = np.exp(log_m)
+    return m * O.logit_variance_estimate(q, summ, scale) / 2 if mode == "compkv" else m
+
+
+def _scores_full_variance(q, summ, scale, mode="compkv"):
+    s = _orig["head_scores"](q, summ, scale, mode)
+    return s * 2 if mode == "compkv" else s
+
+
+def _attn_no_count(q, k, v, summ, selected, scale, block_size=16, compensate=True):
+    saved = summ.count
+    try:
+        summ.count = np.ones_like(saved)
+        # keep the selected blocks' token ranges (they do not use the count)
+        return _orig["compensated_attention"](q, k, v, summ, selected, scale, block_size,
+                                              compensate)
+    finally:
+        summ.count = saved
+
+
+def _attn_shifted_value(q, k, v, summ, selected, scale, block_size=16, compensate=True):
+    saved = summ.mean_v
+    try:
+        summ.mean_v = np.roll(saved, 1, axis=0)
+        return _orig["compensated_attention"](q, k, v, summ, selected, scale, block_size,
+                                              compensate)
+    finally:
+        summ.mean_v = saved
+
+
+def _select_high_ties(S, k_sel):
+    S = np.asarray(S, dtype=float)
+    order = np.lexsort((-np.arange(S.shape[0]), -S))
+    return np.sort(order[:k_sel])
+
+
+def _select_unsorted(S, k_sel):
+    S = np.asarray(S, dtype=float)
+    return np.lexsort((np.arange(S.shape[0]), -S))[:k_sel]
+
+
+def _lbar_sign(q, summ, scale):
+    return -_orig["block_mean_logits"](q, summ, scale)
+
+
+def _dense_scale2(q, k, v, scale):
+    return _orig["dense_attention"](q, k, v, scale * scale)
+
+
+def _group_first_head(q_group, summ, scale, mode="compkv"):
+    q_group = np.atleast_2d(np.asarray(q_group, dtype=float))
+    return O.head_scores(q_group[0], summ, scale, mode)
+
+
+def _logits_no_scale(q, k, scale):
+    return _orig["token_logits"](q, k, 1.0)
+
+
+MUTATIONS = {
+    "sample_variance": ("block_summaries", _summaries_sample_var),
+    "interleaved_groups": ("block_summaries", _summaries_interleaved),
+    "vhat_missing_scale": ("logit_variance_estimate", _vhat_one_scale),
+    "mass_without_second_order": ("second_order_log_mass", _logm_no_second_order),
+    "mass_without_count": ("second_order_log_mass", _logm_no_count),
+    "score_not_normalised": ("head_scores", _scores_unnormalised),
+    "score_full_variance": ("head_scores", _scores_full_variance),
+    "compensation_without_count": ("compensated_attention", _attn_no_count),
+    "compensation_wrong_block_value": ("compensated_attention", _attn_shifted_value),
+    "ties_to_higher_index": ("select_blocks", _select_high_ties),
+    "selection_not_ascending": ("select_blocks", _select_unsorted),
+    "mean_logit_sign": ("block_mean_logits", _lbar_sign),
+    "dense_wrong_scale": ("dense_attention", _dense_scale2),
+    "gqa_first_head_only": ("group_scores", _group_first_head),
+    "logits_without_scale": ("token_logits", _logits_no_scale),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for check in C.ALL_CHECKS:
+        try:
+            check()
+        except (AssertionError, ValueError, IndexError, FloatingPointError) as e:  # noqa: PERF203
+            failed.append(check.__name__)
+        except Exception as e:  # a crash also counts as caught, but say which
+            failed.append(f"{check.__name__}:{type(e).__name__}")
+    assert failed, f"mutation {name} passed every pin"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for check in C.ALL_CHECKS:
+        check()
+    assert math.isfinite(1.0)
