@@ -1,0 +1,352 @@
+// Device helpers shared by the CompKV kernels (sm_100a): mbarrier + bulk-copy pipelines,
+// thread-block-cluster barriers and distributed shared memory, programmatic dependent launch,
+// bf16 unpacking, warp/CTA reductions and an order-preserving float key.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "compkv.h"
+
+namespace compkv {
+
+constexpr int kBlockTokens = 16;      // tokens per KV block
+constexpr int kThreads = 256;         // threads per CTA for every kernel here
+constexpr int kWarps = kThreads / 32;
+
+// ------------------------------------------------------------------------------ addresses
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------------------------------ mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes barrier initialisation visible to the async proxy (bulk copies) and the cluster.
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of a barrier, giving up after a bounded number of attempts (each
+// attempt suspends the thread for a hardware-chosen interval). On giving up it records
+// COMPKV_DEVERR_WAIT_TIMEOUT in *status and returns false; callers then skip the work that
+// needed the data but keep every barrier of the CTA / cluster.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+  for (uint32_t it = 0; it < (1u << 22); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+  }
+  if (status != nullptr) atomicOr(status, COMPKV_DEVERR_WAIT_TIMEOUT);
+  return false;
+}
+
+// Orders this thread's earlier generic-proxy shared-memory writes before later async-proxy
+// (bulk copy) accesses of the same bytes.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------ async copies
+
+// Bulk (non-tensor) copy global -> this CTA's shared memory, completing on `bar` with a
+// transaction count of `bytes`. dst, src and bytes must be multiples of 16 bytes. No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Same, with an L2 evict-first hint for data that is read once per step.
+__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint32_t bytes,
+                                                uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 4-byte asynchronous copy (any 4-byte aligned address); tracked by cp_async_arrive.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+
+// Arrives on `bar` once all of this thread's earlier cp.async copies have landed. The barrier's
+// expected count must include this arrival (noinc).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// ------------------------------------------------------------------------------ clusters
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Full cluster barrier with release/acquire semantics for shared and global memory.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// Address of the same shared variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// ------------------------------------------------------------------------------ PDL
+
+// Blocks until the preceding grid on the stream has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next grid on the stream (launched with programmatic serialisation) start its prologue.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------ numerics
+
+// Unpacks 8 bf16 (one 16-byte word) or 4 fp32 into floats.
+__device__ __forceinline__ void unpack8_bf16(const uint4& w, float (&f)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(u[i] << 16);
+    f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(uint16_t x) {
+  return __uint_as_float(static_cast<uint32_t>(x) << 16);
+}
+
+// Order-preserving map of a non-negative float to uint32 (larger float -> larger key); keys of
+// real scores are >= 0x80000000, so key 0 ranks below every real score.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  const uint32_t b = __float_as_uint(s);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// exp(a - b) that treats (-inf) - (-inf) as an empty term (0) instead of NaN.
+__device__ __forceinline__ float exp_diff(float a, float b) {
+  return (a == -CUDART_INF_F) ? 0.f : __expf(a - b);
+}
+
+// Online log-sum-exp pair (max, sum of exp(x - max)); merges another pair.
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  if (m2 == -CUDART_INF_F) return;
+  if (m == -CUDART_INF_F) {
+    m = m2;
+    s = s2;
+    return;
+  }
+  const float mn = fmaxf(m, m2);
+  s = s * __expf(m - mn) + s2 * __expf(m2 - mn);
+  m = mn;
+}
+
+// ------------------------------------------------------------------------------ CTA helpers
+
+// Exclusive prefix sum of one int per thread over the CTA; also returns the total.
+// `sh` needs kWarps + 1 ints. Contains __syncthreads.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* sh, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sh[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < kWarps) ? sh[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    if (lane < kWarps) sh[lane] = wi - w;
+    if (lane == kWarps - 1) sh[kWarps] = wi;
+  }
+  __syncthreads();
+  const int res = sh[warp] + incl - v;
+  total = sh[kWarps];
+  __syncthreads();
+  return res;
+}
+
+// Radix select over 32-bit keys: the K-th largest key value tau (1 <= K <= n) and the number of
+// keys strictly greater than tau. 8-bit digits, most significant first. `hist` holds 256 uints,
+// `bc` 2 uints. All threads call it; all get the result. Contains __syncthreads.
+template <typename KeyAt>
+__device__ void cta_radix_select(KeyAt key_at, int n, int K, uint32_t* hist, uint32_t* bc,
+                                 uint32_t& tau, int& n_greater) {
+  uint32_t prefix = 0, pmask = 0;
+  uint32_t k = static_cast<uint32_t>(K);
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const uint32_t key = key_at(i);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x;
+      uint32_t c[8], tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        c[e] = hist[255 - 8 * lane - e];
+        tot += c[e];
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const uint32_t excl = incl - tot;
+      if (excl < k && k <= incl) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (run + c[e] >= k) {
+            bc[0] = static_cast<uint32_t>(255 - 8 * lane - e);
+            bc[1] = k - run;
+            break;
+          }
+          run += c[e];
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = bc[0];
+    k = bc[1];
+    prefix |= bin << shift;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  tau = prefix;
+  n_greater = K - static_cast<int>(k);
+}
+
+// Stable selection of the top-K under (key desc, index asc) given tau and n_greater from
+// cta_radix_select: item i is kept if key > tau, or key == tau and fewer than K - n_greater
+// equal keys precede it. Kept items are visited in index order with their output position:
+// emit(i, pos). `sh` needs kWarps + 1 ints. Contains __syncthreads. Returns the number kept.
+template <typename KeyAt, typename Emit>
+__device__ int cta_select_ordered(KeyAt key_at, int n, int K, uint32_t tau, int n_greater,
+                                  int* sh, Emit emit) {
+  const int per = (n + kThreads - 1) / kThreads;
+  const int i0 = min(n, static_cast<int>(threadIdx.x) * per), i1 = min(n, i0 + per);
+  int eq = 0;
+  for (int i = i0; i < i1; ++i) eq += (key_at(i) == tau);
+  int eq_total;
+  const int eq_before = cta_exclusive_scan(eq, sh, eq_total);
+  const int quota = K - n_greater;
+  int kept = 0, er = eq_before;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t key = key_at(i);
+    if (key > tau) {
+      ++kept;
+    } else if (key == tau) {
+      if (er < quota) ++kept;
+      ++er;
+    }
+  }
+  int kept_total;
+  int pos = cta_exclusive_scan(kept, sh, kept_total);
+  er = eq_before;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t key = key_at(i);
+    bool keep = false;
+    if (key > tau) {
+      keep = true;
+    } else if (key == tau) {
+      keep = er < quota;
+      ++er;
+    }
+    if (keep) emit(i, pos++);
+  }
+  return kept_total;
+}
+
+}  // namespace compkv
