@@ -2,19 +2,20 @@
 // dispatch. No allocation, no host synchronisation (except compkv_read_device_status).
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
-#include <string>
 
 #include "compkv.h"
 #include "internal.h"
 
 namespace {
 
-thread_local std::string g_last_cuda_error;
+thread_local char g_last_cuda_error[256] = "";
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return COMPKV_OK;
-  g_last_cuda_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
   return COMPKV_ERR_CUDA;
 }
 
@@ -61,14 +62,14 @@ float scale_of(const compkv_shape* s, float softmax_scale) {
   return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(s->head_dim));
 }
 
-size_t comp_bytes(const compkv_shape* s) {
-  const int G = s->n_q_heads / s->n_kv_heads;
-  return compkv::align256(sizeof(float) * static_cast<size_t>(s->batch) * s->n_kv_heads *
-                          compkv::comp_partial_floats(G, s->head_dim));
+compkv::StepWorkspace step_ws(const compkv_shape* s) {
+  compkv::StepWorkspace w;
+  w.build(s->batch * s->n_kv_heads, n_blocks(s), s->n_q_heads / s->n_kv_heads, s->head_dim);
+  return w;
 }
 
 int32_t* status_word(void* ws) { return static_cast<int32_t*>(ws); }
-float* comp_area(void* ws) { return reinterpret_cast<float*>(static_cast<char*>(ws) + compkv::kWsHeader); }
+float* ws_at(void* ws, size_t off) { return reinterpret_cast<float*>(static_cast<char*>(ws) + off); }
 
 struct Common {
   int G, Nb, Kb;
@@ -104,7 +105,7 @@ int32_t compkv_num_selected(const compkv_shape* shape, int32_t budget_tokens) {
 
 size_t compkv_workspace_bytes(const compkv_shape* shape, int32_t budget_tokens) {
   if (check_shape(shape) != COMPKV_OK || budget_tokens < 0) return 0;
-  return compkv::kWsHeader + comp_bytes(shape);
+  return step_ws(shape).total;
 }
 
 size_t compkv_full_workspace_bytes(const compkv_shape* shape) {
@@ -159,27 +160,48 @@ static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, comp
   if (!aligned16(q) || !aligned16(mean_k) || (comp && !aligned16(mean_v)) || !aligned4(var_g) ||
       !aligned4(count) || (sel_idx && !aligned4(sel_idx)) || (scores && !aligned4(scores)))
     return COMPKV_ERR_BAD_ALIGNMENT;
-  compkv::ScoreSelectArgs a;
+  const compkv::StepWorkspace W = step_ws(shape);
+  const int pairs = shape->batch * shape->n_kv_heads;
+  int nctas = 0;
+  compkv::StreamArgs a;
   a.bf16 = dtype == COMPKV_BF16;
   a.mode = mode;
-  a.B = shape->batch;
-  a.Hkv = shape->n_kv_heads;
+  a.pairs = pairs;
   a.G = c.G;
   a.D = shape->head_dim;
   a.Nb = c.Nb;
   a.r = shape->n_groups;
-  a.Kb = c.Kb;
+  a.slots = W.slots;
   a.scale = scale_of(shape, softmax_scale);
   a.q = q;
   a.mean_k = mean_k;
   a.var_g = var_g;
   a.mean_v = mean_v;
   a.count = count;
-  a.sel_idx = sel_idx;
-  a.scores = scores;
-  a.comp = comp_area(workspace);
+  a.u = ws_at(workspace, W.u);
+  a.zpart = ws_at(workspace, W.zpart);
+  a.comp_seg = ws_at(workspace, W.comp_seg);
   a.status = status_word(workspace);
-  return cuda_status(compkv::launch_score_select(a, static_cast<cudaStream_t>(stream)));
+  a.nctas_out = &nctas;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int rc = cuda_status(compkv::launch_score_stream(a, cs));
+  if (rc) return rc;
+  compkv::SelectArgs b;
+  b.mode = mode;
+  b.pairs = pairs;
+  b.G = c.G;
+  b.D = shape->head_dim;
+  b.Nb = c.Nb;
+  b.Kb = c.Kb;
+  b.slots = W.slots;
+  b.nctas_stream = nctas;
+  b.u = a.u;
+  b.zpart = a.zpart;
+  b.comp_seg = a.comp_seg;
+  b.comp = ws_at(workspace, W.comp);
+  b.sel_idx = sel_idx;
+  b.scores = scores;
+  return cuda_status(compkv::launch_select(b, cs));
 }
 
 static int sparse_decode_impl(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
@@ -214,7 +236,7 @@ static int sparse_decode_impl(const compkv_shape* shape, compkv_dtype dtype, com
   a.mean_v = mean_v;
   a.count = count;
   a.sel_idx = sel_idx;
-  a.comp = comp_area(workspace);
+  a.comp = ws_at(workspace, step_ws(shape).comp);
   a.out = out;
   a.status = status_word(workspace);
   a.pdl = pdl;
@@ -314,7 +336,7 @@ const char* compkv_status_string(int status) {
   }
 }
 
-const char* compkv_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+const char* compkv_last_cuda_error(void) { return g_last_cuda_error; }
 
 int compkv_version(void) { return COMPKV_VERSION; }
 

@@ -252,29 +252,39 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* sh, int& total) {
   return res;
 }
 
-// Radix select over 32-bit keys: the K-th largest key value tau (1 <= K <= n) and the number of
-// keys strictly greater than tau. 8-bit digits, most significant first. `hist` holds 256 uints,
-// `bc` 2 uints. All threads call it; all get the result. Contains __syncthreads.
+// Top-K threshold by most-significant-digit radix select over 32-bit keys (8-bit digits).
+// Finds the bucket (prefix under mask) that holds the K-th largest key (1 <= K <= n) and the
+// number `quota` of keys in that bucket that belong to the top K; keys in higher buckets all
+// belong. Stops early once the whole bucket is selected. `hist` holds 2 x 256 uints, `bc` 4
+// uints. All threads call it and get the result; two CTA barriers per digit.
+struct RadixCut {
+  uint32_t prefix, mask;
+  int quota;
+};
+
 template <typename KeyAt>
-__device__ void cta_radix_select(KeyAt key_at, int n, int K, uint32_t* hist, uint32_t* bc,
-                                 uint32_t& tau, int& n_greater) {
-  uint32_t prefix = 0, pmask = 0;
+__device__ RadixCut cta_radix_cut(KeyAt key_at, int n, int K, uint32_t* hist, uint32_t* bc) {
+  uint32_t prefix = 0, mask = 0;
   uint32_t k = static_cast<uint32_t>(K);
+  for (int i = threadIdx.x; i < 512; i += kThreads) hist[i] = 0;
+  __syncthreads();
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
-    __syncthreads();
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    uint32_t* H = hist + (pass & 1) * 256;
+    uint32_t* Hn = hist + ((pass + 1) & 1) * 256;
     for (int i = threadIdx.x; i < n; i += kThreads) {
       const uint32_t key = key_at(i);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&H[(key >> shift) & 255u], 1u);
     }
+    for (int i = threadIdx.x; i < 256; i += kThreads) Hn[i] = 0;
     __syncthreads();
     if (threadIdx.x < 32) {
       const int lane = threadIdx.x;
       uint32_t c[8], tot = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        c[e] = hist[255 - 8 * lane - e];
+        c[e] = H[255 - 8 * lane - e];
         tot += c[e];
       }
       uint32_t incl = tot;
@@ -291,6 +301,7 @@ __device__ void cta_radix_select(KeyAt key_at, int n, int K, uint32_t* hist, uin
           if (run + c[e] >= k) {
             bc[0] = static_cast<uint32_t>(255 - 8 * lane - e);
             bc[1] = k - run;
+            bc[2] = c[e];
             break;
           }
           run += c[e];
@@ -298,50 +309,39 @@ __device__ void cta_radix_select(KeyAt key_at, int n, int K, uint32_t* hist, uin
       }
     }
     __syncthreads();
-    const uint32_t bin = bc[0];
+    const uint32_t bin = bc[0], cnt = bc[2];
     k = bc[1];
     prefix |= bin << shift;
-    pmask |= 255u << shift;
-    __syncthreads();
+    mask |= 255u << shift;
+    if (cnt == k) break;  // every key of the bucket is in the top K
   }
-  tau = prefix;
-  n_greater = K - static_cast<int>(k);
+  return RadixCut{prefix, mask, static_cast<int>(k)};
 }
 
-// Stable selection of the top-K under (key desc, index asc) given tau and n_greater from
-// cta_radix_select: item i is kept if key > tau, or key == tau and fewer than K - n_greater
-// equal keys precede it. Kept items are visited in index order with their output position:
-// emit(i, pos). `sh` needs kWarps + 1 ints. Contains __syncthreads. Returns the number kept.
+// Keeps item i if (key & mask) > prefix, or it equals prefix and fewer than `quota` such items
+// precede it; visits kept items in index order with their output position: emit(i, pos).
+// `sh` needs kWarps + 1 ints. Contains CTA barriers. Returns the number kept.
 template <typename KeyAt, typename Emit>
-__device__ int cta_select_ordered(KeyAt key_at, int n, int K, uint32_t tau, int n_greater,
-                                  int* sh, Emit emit) {
+__device__ int cta_select_ordered(KeyAt key_at, int n, const RadixCut& cut, int* sh, Emit emit) {
   const int per = (n + kThreads - 1) / kThreads;
   const int i0 = min(n, static_cast<int>(threadIdx.x) * per), i1 = min(n, i0 + per);
-  int eq = 0;
-  for (int i = i0; i < i1; ++i) eq += (key_at(i) == tau);
+  int eq = 0, gt = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t km = key_at(i) & cut.mask;
+    eq += (km == cut.prefix);
+    gt += (km > cut.prefix);
+  }
   int eq_total;
   const int eq_before = cta_exclusive_scan(eq, sh, eq_total);
-  const int quota = K - n_greater;
-  int kept = 0, er = eq_before;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    if (key > tau) {
-      ++kept;
-    } else if (key == tau) {
-      if (er < quota) ++kept;
-      ++er;
-    }
-  }
+  const int kept_eq = max(0, min(eq, cut.quota - eq_before));
   int kept_total;
-  int pos = cta_exclusive_scan(kept, sh, kept_total);
-  er = eq_before;
+  int pos = cta_exclusive_scan(gt + kept_eq, sh, kept_total);
+  int er = eq_before;
   for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    bool keep = false;
-    if (key > tau) {
-      keep = true;
-    } else if (key == tau) {
-      keep = er < quota;
+    const uint32_t km = key_at(i) & cut.mask;
+    bool keep = km > cut.prefix;
+    if (km == cut.prefix) {
+      keep = er < cut.quota;
       ++er;
     }
     if (keep) emit(i, pos++);

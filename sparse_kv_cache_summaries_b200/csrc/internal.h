@@ -10,6 +10,8 @@
 namespace compkv {
 
 constexpr int kBlockTokensHost = 16;  // the only supported block size
+constexpr int kStreamTile = 32;       // blocks per tile of the streaming score kernel
+constexpr int kStreamMaxCtas = 384;   // grid cap of the streaming score kernel
 
 struct SummariesArgs {
   bool bf16;
@@ -23,24 +25,36 @@ struct SummariesArgs {
   int32_t* count;
 };
 
-// Per-kv-head Mean-compensation partial, merged over all blocks: [m, l, acc[D]] per query head.
-// m is the running max of (lbar + log n), l = sum n e^{lbar - m}, acc = sum n e^{lbar - m} nu.
+// A Mean-compensation partial per query head: [m, l, acc[D]] with m a reference logit,
+// l = sum n e^{lbar - m} and acc = sum n e^{lbar - m} nu over the blocks it covers.
 inline size_t comp_partial_floats(int G, int D) { return static_cast<size_t>(G) * (D + 2); }
 
-struct ScoreSelectArgs {
+struct StreamArgs {
   bool bf16;
   int mode;
-  int B, Hkv, G, D, Nb, r, Kb;
+  int pairs, G, D, Nb, r, slots;
   float scale;
   const void* q;
   const float* mean_k;
   const float* var_g;
   const float* mean_v;
   const int32_t* count;
-  int32_t* sel_idx;
-  float* scores;
-  float* comp;        // [B*Hkv][G][D+2]
-  int32_t* status;    // device status word
+  float* u;          // [pairs][Nb][G]   per-block log scores
+  float* zpart;      // [pairs][slots][G][2]   log-sum-exp partials of the mass estimate
+  float* comp_seg;   // [pairs][slots][G][D+2] compensation partials per segment
+  int32_t* status;
+  int* nctas_out;    // grid size used (host), may be null
+};
+
+struct SelectArgs {
+  int mode;
+  int pairs, G, D, Nb, Kb, slots, nctas_stream;
+  const float* u;
+  const float* zpart;
+  const float* comp_seg;
+  float* comp;       // [pairs][G][D+2] merged compensation partial
+  int32_t* sel_idx;  // [pairs][Kb]
+  float* scores;     // [pairs][Nb] or null
 };
 
 struct SparseArgs {
@@ -55,10 +69,10 @@ struct SparseArgs {
   const float* mean_v;
   const int32_t* count;
   const int32_t* sel_idx;
-  const float* comp;  // [B*Hkv][G][D+2] from score_select
+  const float* comp;  // [B*Hkv][G][D+2] merged compensation partial
   float* out;
   int32_t* status;
-  bool pdl;           // launched right after score_select: use programmatic dependent launch
+  bool pdl;           // launched right after the select kernel: programmatic dependent launch
 };
 
 struct FullArgs {
@@ -76,15 +90,38 @@ struct FullArgs {
   int32_t* status;
 };
 
-// Workspace layout (bytes, 256-aligned sections):
-//   [0, 256)            int32 status word
-//   comp partials       B*Hkv*G*(D+2) floats
-constexpr size_t kWsHeader = 256;
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+constexpr size_t kWsHeader = 256;
 
-// Cluster size used by score_select for this shape on the current device (1..16).
-int score_select_cluster(int B, int Hkv, int G, int D, int r, int Nb, int Kb, bool bf16,
-                         size_t* smem_bytes);
+// Segment records per (sequence, kv-head) the streaming kernel may write: the tiles_per_pair
+// tiles of a pair meet at most ceil(tiles_per_pair / min_tiles_per_cta) + 1 CTA ranges, and a
+// grid of at most kStreamMaxCtas CTAs gives every CTA at least floor(F / kStreamMaxCtas) tiles.
+inline int stream_slots(int pairs, int Nb) {
+  const long long tp = (Nb + kStreamTile - 1) / kStreamTile;
+  const long long F = tp * pairs;
+  long long min_tiles = F / kStreamMaxCtas;
+  if (min_tiles < 1) min_tiles = 1;
+  return static_cast<int>((tp + min_tiles - 1) / min_tiles + 1);
+}
+
+// Workspace of the sparse step: a 256-byte header whose first int32 is the device status word,
+// then 256-aligned sections.
+struct StepWorkspace {
+  size_t u, zpart, comp_seg, comp, total;
+  int slots;
+  void build(int pairs, int Nb, int G, int D) {
+    slots = stream_slots(pairs, Nb);
+    size_t o = kWsHeader;
+    u = o;        o += align256(sizeof(float) * static_cast<size_t>(pairs) * Nb * G);
+    zpart = o;    o += align256(sizeof(float) * static_cast<size_t>(pairs) * slots * G * 2);
+    comp_seg = o; o += align256(sizeof(float) * static_cast<size_t>(pairs) * slots * G * (D + 2));
+    comp = o;     o += align256(sizeof(float) * static_cast<size_t>(pairs) * comp_partial_floats(G, D));
+    total = o;
+  }
+};
+
+// Grid size of the streaming score kernel for this shape on the current device.
+int stream_grid_ctas(bool bf16, int D, int G, int r, int total_tiles);
 // Blocks per CTA and the CTA count per kv-head (a cluster) of sparse_decode.
 void sparse_split(int B, int Hkv, int Kb, int* blocks_per_cta, int* nsplit);
 // Splits per kv-head of full_decode (<= max_full_splits(T)).
@@ -92,7 +129,8 @@ int full_splits(int B, int Hkv, int T);
 inline int max_full_splits(int T) { return (T + 511) / 512; }
 
 cudaError_t launch_build_summaries(const SummariesArgs& a, cudaStream_t st);
-cudaError_t launch_score_select(const ScoreSelectArgs& a, cudaStream_t st);
+cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_decode(const SparseArgs& a, cudaStream_t st);
 cudaError_t launch_full_decode(const FullArgs& a, cudaStream_t st);
 

@@ -16,9 +16,13 @@
 // partials (m, l, acc) are merged by rank 0 over DSMEM together with the compensation partial.
 // Launched with programmatic dependent launch after the score kernel: the q prologue runs before
 // griddepcontrol.wait, everything that reads the selection after it.
+#include <cooperative_groups.h>
+
 #include "attend.cuh"
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace compkv {
 namespace {
@@ -54,7 +58,7 @@ struct SLayout {
   static constexpr size_t off_ml = off_acc + sizeof(float) * G * D;      // [G][2]
   static constexpr size_t off_blk = off_ml + sizeof(float) * 2 * 8;      // j, n, slot flags
   static constexpr size_t off_lbar = off_blk + sizeof(int) * 2 * kRound; // [G][kRound]
-  static constexpr size_t off_pw = off_lbar + sizeof(float) * G * kRound;
+  static constexpr size_t off_pw = off_lbar + sizeof(float) * G * 17;
   static constexpr size_t off_sc = off_pw + sizeof(float) * G * kRound;  // [G]
   static constexpr size_t off_fac = off_sc + sizeof(float) * 8;          // [G][17]
   static constexpr size_t off_mbar = (off_fac + sizeof(float) * G * 17 + 15) & ~size_t(15);
@@ -263,20 +267,24 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
   cluster_sync();  // #1: every split's partial is visible
 
   if (rank == 0) {
+    cg::cluster_group cluster = cg::this_cluster();
     const float* cp = p.comp + static_cast<size_t>(bk) * G * (D + 2);
     // per head: common max over the splits and the compensation partial, factors, 1/denominator
     if (tid < G * NS) {
       const int h = tid / NS, s = tid % NS;
-      fac_s[h * 17 + s] = ld_dsmem_f32(dsmem_addr(&ml_s[2 * h], s));
+      const float* rml = cluster.map_shared_rank(ml_s, s);
+      fac_s[h * 17 + s] = rml[2 * h];
+      lbar_s[h * 17 + s] = rml[2 * h + 1];   // reused as scratch for the split denominators
     }
     __syncthreads();
     if (tid < G) {
       const int h = tid;
-      float M = compensate ? cp[h * (D + 2)] : -CUDART_INF_F;
+      const float cm = compensate ? cp[h * (D + 2)] : -CUDART_INF_F;
+      float M = cm;
       for (int s = 0; s < NS; ++s) M = fmaxf(M, fac_s[h * 17 + s]);
       float den = 0.f;
-      if (compensate && cp[h * (D + 2)] != -CUDART_INF_F) {
-        const float f = __expf(cp[h * (D + 2)] - M);
+      if (cm != -CUDART_INF_F) {
+        const float f = __expf(cm - M);
         fac_s[h * 17 + 16] = f;
         den = f * cp[h * (D + 2) + 1];
       } else {
@@ -286,7 +294,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
         const float ms = fac_s[h * 17 + s];
         const float f = (ms == -CUDART_INF_F) ? 0.f : __expf(ms - M);
         fac_s[h * 17 + s] = f;
-        den = fmaf(f, ld_dsmem_f32(dsmem_addr(&ml_s[2 * h + 1], s)), den);
+        den = fmaf(f, lbar_s[h * 17 + s], den);
       }
       sc_s[h] = den > 0.f ? 1.f / den : 0.f;
     }
@@ -294,8 +302,12 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
     float* o = p.out + static_cast<size_t>(bk) * G * D;
     for (int i = tid; i < G * D; i += kThreads) {
       const int h = i / D, c = i % D;
+      float part[16];
+#pragma unroll
+      for (int s = 0; s < 16; ++s) part[s] = (s < NS) ? cluster.map_shared_rank(acc_s, s)[i] : 0.f;
       float a = compensate ? fac_s[h * 17 + 16] * cp[h * (D + 2) + 2 + c] : 0.f;
-      for (int s = 0; s < NS; ++s) a = fmaf(fac_s[h * 17 + s], ld_dsmem_f32(dsmem_addr(&acc_s[i], s)), a);
+#pragma unroll
+      for (int s = 0; s < 16; ++s) a = fmaf(fac_s[h * 17 + s], part[s], a);
       o[i] = a * sc_s[h];
     }
   }
