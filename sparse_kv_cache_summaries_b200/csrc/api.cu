@@ -179,6 +179,7 @@ static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, comp
   a.mean_v = mean_v;
   a.count = count;
   a.u = ws_at(workspace, W.u);
+  a.xrec = ws_at(workspace, W.xrec);
   a.zpart = ws_at(workspace, W.zpart);
   a.comp_seg = ws_at(workspace, W.comp_seg);
   a.status = status_word(workspace);
@@ -237,6 +238,7 @@ static int sparse_decode_impl(const compkv_shape* shape, compkv_dtype dtype, com
   a.count = count;
   a.sel_idx = sel_idx;
   a.comp = ws_at(workspace, step_ws(shape).comp);
+  a.xrec = ws_at(workspace, step_ws(shape).xrec);
   a.out = out;
   a.status = status_word(workspace);
   a.pdl = pdl;

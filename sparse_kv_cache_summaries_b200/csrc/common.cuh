@@ -273,9 +273,15 @@ __device__ RadixCut cta_radix_cut(KeyAt key_at, int n, int K, uint32_t* hist, ui
     const int shift = 24 - 8 * pass;
     uint32_t* H = hist + (pass & 1) * 256;
     uint32_t* Hn = hist + ((pass + 1) & 1) * 256;
-    for (int i = threadIdx.x; i < n; i += kThreads) {
-      const uint32_t key = key_at(i);
-      if ((key & mask) == prefix) atomicAdd(&H[(key >> shift) & 255u], 1u);
+    // warp-aggregated counting: one atomic per distinct digit per warp (float keys crowd into a
+    // few top-digit buckets, where plain per-key atomics serialise)
+    const int n32 = (n + 31) & ~31;
+    for (int i = threadIdx.x; i < n32; i += kThreads) {
+      const uint32_t key = i < n ? key_at(i) : 0u;
+      const bool m = i < n && (key & mask) == prefix;
+      const uint32_t bin = (key >> shift) & 255u;
+      const uint32_t grp = __match_any_sync(0xffffffffu, m ? bin : 256u + (threadIdx.x & 31));
+      if (m && (__ffs(grp) - 1) == static_cast<int>(threadIdx.x & 31)) atomicAdd(&H[bin], __popc(grp));
     }
     for (int i = threadIdx.x; i < 256; i += kThreads) Hn[i] = 0;
     __syncthreads();

@@ -13,6 +13,10 @@ constexpr int kBlockTokensHost = 16;  // the only supported block size
 constexpr int kStreamTile = 32;       // blocks per tile of the streaming score kernel
 constexpr int kStreamMaxCtas = 384;   // grid cap of the streaming score kernel
 
+// Floats per block of the record {x_0..x_{G-1}, n} the streaming kernel writes for the attention
+// kernel (x_h = s q_h . mu_j + log n_j; n as int bits), padded to 16 bytes.
+__host__ __device__ constexpr int xrec_stride(int G) { return ((G + 1 + 3) / 4) * 4; }
+
 struct SummariesArgs {
   bool bf16;
   int B, Hkv, T, D, Nb, r;
@@ -40,6 +44,7 @@ struct StreamArgs {
   const float* mean_v;
   const int32_t* count;
   float* u;          // [pairs][Nb][G]   per-block log scores
+  float* xrec;       // [pairs][Nb][xrec_stride(G)]
   float* zpart;      // [pairs][slots][G][2]   log-sum-exp partials of the mass estimate
   float* comp_seg;   // [pairs][slots][G][D+2] compensation partials per segment
   int32_t* status;
@@ -70,6 +75,7 @@ struct SparseArgs {
   const int32_t* count;
   const int32_t* sel_idx;
   const float* comp;  // [B*Hkv][G][D+2] merged compensation partial
+  const float* xrec;  // [B*Hkv][Nb][xrec_stride(G)] from the streaming kernel
   float* out;
   int32_t* status;
   bool pdl;           // launched right after the select kernel: programmatic dependent launch
@@ -107,12 +113,13 @@ inline int stream_slots(int pairs, int Nb) {
 // Workspace of the sparse step: a 256-byte header whose first int32 is the device status word,
 // then 256-aligned sections.
 struct StepWorkspace {
-  size_t u, zpart, comp_seg, comp, total;
+  size_t u, xrec, zpart, comp_seg, comp, total;
   int slots;
   void build(int pairs, int Nb, int G, int D) {
     slots = stream_slots(pairs, Nb);
     size_t o = kWsHeader;
     u = o;        o += align256(sizeof(float) * static_cast<size_t>(pairs) * Nb * G);
+    xrec = o;     o += align256(sizeof(float) * static_cast<size_t>(pairs) * Nb * xrec_stride(G));
     zpart = o;    o += align256(sizeof(float) * static_cast<size_t>(pairs) * slots * G * 2);
     comp_seg = o; o += align256(sizeof(float) * static_cast<size_t>(pairs) * slots * G * (D + 2));
     comp = o;     o += align256(sizeof(float) * static_cast<size_t>(pairs) * comp_partial_floats(G, D));

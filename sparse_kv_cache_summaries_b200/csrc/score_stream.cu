@@ -11,18 +11,21 @@
 // Work split (B200): the (sequence, kv-head) tiles of 32 blocks are laid end to end and cut into
 // equal contiguous ranges, one per CTA, two CTAs per SM, so every SM streams the same number of
 // bytes whatever B and Hkv are. A CTA's range crosses at most a few (sequence, kv-head) pairs; it
-// writes one partial record per pair it touches ("segment"). The mean keys and mean values of a
-// tile arrive by bulk copy and the grouped variances and counts by 4-byte cp.async, on one
-// mbarrier per stage of a 3-deep ring.
+// writes one partial record per pair it touches ("segment").
 //
-// Per tile there is one CTA barrier. The D/8 lanes of a block dot its mean key with the G heads
-// (transpose-reduce); the lane that ends up holding head h's dot does the scalar work for that
-// (block, head) and keeps its own running Zhat and compensation sums. Compensation weights use a
-// reference m_ref per head that only moves up when a logit would exceed it by 64 (e^64 keeps
-// every sum finite in fp32), so the common tile needs no max-reduction; the rare tile that moves
-// it takes one extra barrier. Weights go through a double-buffered shared array to the
-// accumulation, where each thread owns 4 channels of all G heads, so each mean value is read
-// from shared memory once.
+// Pipeline: a 3-stage shared-memory ring with a "full" and an "empty" mbarrier per stage. Warp 0
+// refills a stage (bulk copies of the tile's mean keys and mean values, 4-byte cp.async of its
+// grouped variances and counts) once all 8 warps have released it. Each warp owns 4 blocks of
+// every tile and works through the ring on its own, with no CTA barrier in steady state: its
+// lanes dot the mean keys with the G heads (transpose-reduce), the lane left holding head h's dot
+// does that (block, head)'s scalar work, and the warp accumulates its blocks' weighted mean
+// values for all G heads (4 channels per lane). Compensation weights are taken against a
+// per-warp reference logit per head that only moves up when a logit would exceed it by 64 (e^64
+// keeps every sum finite in fp32). Warps meet only where a segment ends, to merge their partials
+// in a fixed order (deterministic results).
+//
+// Besides the log scores u it writes, per block, the record {x_h (h < G), n_j} that lets the
+// attention kernel add and remove the block's compensation term without re-reading its summary.
 #include <mutex>
 
 #include "attend.cuh"
@@ -34,6 +37,7 @@ namespace {
 
 constexpr int kTile = kStreamTile;
 constexpr int kStages = 3;
+constexpr int kBlocksPerWarp = kTile / kWarps;  // 4
 constexpr float kRefSlack = 64.f;
 
 struct StreamParams {
@@ -45,6 +49,7 @@ struct StreamParams {
   const float* mean_v;
   const int32_t* count;
   float* u;        // [pairs][Nb][G]
+  float* xrec;     // [pairs][Nb][xrec_stride(G)]  {x_0..x_{G-1}, n}
   float* zpart;    // [pairs][slots][G][2]
   float* comp;     // [pairs][slots][G][D+2]
   int32_t* status;
@@ -53,7 +58,7 @@ struct StreamParams {
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 struct SLay {
-  size_t stage_bytes, off_mu, off_nu, off_var, off_cnt, stage0, mbar, ws, q, qn, comp, red, misc, total;
+  size_t stage_bytes, off_mu, off_nu, off_var, off_cnt, stage0, full, empty, wsw, q, qn, comp, refw, red, logn, total;
   __host__ __device__ void build(int D, int G, int r) {
     off_mu = 0;
     off_nu = a16(sizeof(float) * kTile * D);
@@ -61,24 +66,27 @@ struct SLay {
     off_cnt = a16(off_var + sizeof(float) * kTile * r);
     stage_bytes = a16(off_cnt + sizeof(int) * kTile);
     size_t o = 0;
-    mbar = o;   o = a16(o + 8 * kStages);
+    full = o;   o = a16(o + 8 * kStages);
+    empty = o;  o = a16(o + 8 * kStages);
     stage0 = o; o = a16(o + stage_bytes * kStages);
-    ws = o;     o = a16(o + sizeof(float) * 2 * kTile * G);   // double-buffered weights [2][kTile][G]
+    wsw = o;    o = a16(o + sizeof(float) * kWarps * kBlocksPerWarp * G);   // per-warp weights
     q = o;      o = a16(o + sizeof(float) * G * D);
     qn = o;     o = a16(o + sizeof(float) * G * r);
     comp = o;   o = a16(o + sizeof(float) * G * D);
-    red = o;    o = a16(o + sizeof(float) * 3 * G * 64);      // per-head lane-slot reductions
-    misc = o;   o = a16(o + sizeof(float) * 64);   // mref[8] sc[8] tmax[3][8] flag[3] logn[17]
+    refw = o;   o = a16(o + sizeof(float) * kWarps * G);
+    red = o;    o = a16(o + sizeof(float) * 3 * G * 32);
+    logn = o;   o = a16(o + sizeof(float) * 17);
     total = o;
   }
 };
 
-// Ordered int of a float (monotone), for shared-memory atomicMax.
-__device__ __forceinline__ int ord_float(float f) {
-  const int i = __float_as_int(f);
-  return i >= 0 ? i : i ^ 0x7fffffff;
+template <int G>
+__device__ __forceinline__ float pick_h(const float (&a)[G], int h) {
+  float v = a[0];
+#pragma unroll
+  for (int i = 1; i < G; ++i) v = (h == i) ? a[i] : v;
+  return v;
 }
-__device__ __forceinline__ float unord_float(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
 template <typename TQ, int D, int G>
 __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_constant__ StreamParams p) {
@@ -92,22 +100,21 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   const int f0 = static_cast<int>((static_cast<long long>(blockIdx.x) * F) / p.nctas);
   const int f1 = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * F) / p.nctas);
   const int nt = f1 - f0;
+  constexpr int XS = xrec_stride(G);
 
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L.mbar);
-  float* ws_s = reinterpret_cast<float*>(sm + L.ws);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.full);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(sm + L.empty);
+  float* wsw = reinterpret_cast<float*>(sm + L.wsw) + warp * kBlocksPerWarp * G;
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   float* qn_s = reinterpret_cast<float*>(sm + L.qn);
   float* comp_s = reinterpret_cast<float*>(sm + L.comp);
+  float* refw_s = reinterpret_cast<float*>(sm + L.refw);
   float* red_s = reinterpret_cast<float*>(sm + L.red);
-  float* mref_s = reinterpret_cast<float*>(sm + L.misc);        // [8] compensation reference
-  float* sc_s = mref_s + 8;                                       // [8] rescale factors
-  int* tmax_s = reinterpret_cast<int*>(mref_s + 16);              // [3][8] tile max (ordered)
-  int* flag_s = tmax_s + 24;                                      // [3]
-  float* logn_s = mref_s + 44;                                    // [17]
+  float* logn_s = reinterpret_cast<float*>(sm + L.logn);
   const uint64_t policy = l2_evict_first_policy();
 
-  auto tile_pair = [&](int f) { return f / TP; };
-  auto issue = [&](int k) {  // local tile k -> stage k % kStages
+  // Refills the stage of local tile k (warp 0 only; all 32 lanes).
+  auto issue = [&](int k) {
     const int f = f0 + k;
     const int pr = f / TP, t = f % TP;
     const int jt0 = t * kTile;
@@ -117,77 +124,103 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     unsigned char* sb = sm + L.stage0 + L.stage_bytes * st;
     float* var_d = reinterpret_cast<float*>(sb + L.off_var);
     int* cnt_d = reinterpret_cast<int*>(sb + L.off_cnt);
-    for (int i = tid; i < tn * r; i += kThreads) cp_async4(var_d + i, p.var_g + row0 * r + i);
-    for (int i = tid; i < tn; i += kThreads) cp_async4(cnt_d + i, p.count + row0 + i);
-    if (tid == 0) {
+    for (int i = lane; i < tn * r; i += 32) cp_async4(var_d + i, p.var_g + row0 * r + i);
+    for (int i = lane; i < tn; i += 32) cp_async4(cnt_d + i, p.count + row0 + i);
+    if (lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>(tn) * D * sizeof(float);
-      mbar_arrive_expect_tx(&mbar[st], compensate ? 2 * bytes : bytes);
-      bulk_g2s_stream(sb + L.off_mu, p.mean_k + row0 * D, bytes, &mbar[st], policy);
-      if (compensate) bulk_g2s_stream(sb + L.off_nu, p.mean_v + row0 * D, bytes, &mbar[st], policy);
+      mbar_arrive_expect_tx(&full[st], compensate ? 2 * bytes : bytes);
+      bulk_g2s_stream(sb + L.off_mu, p.mean_k + row0 * D, bytes, &full[st], policy);
+      if (compensate) bulk_g2s_stream(sb + L.off_nu, p.mean_v + row0 * D, bytes, &full[st], policy);
     }
-    cp_async_arrive(&mbar[st]);
+    cp_async_arrive(&full[st]);
   };
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], kThreads + 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 32 + 1);
+      mbar_init(&empty[s], kWarps);
+    }
     mbar_init_fence();
   }
   if (tid < 17) logn_s[tid] = tid > 0 ? logf(static_cast<float>(tid)) : -CUDART_INF_F;
   __syncthreads();
-  for (int k = 0; k < min(nt, kStages - 1); ++k) issue(k);
+  int issued = min(nt, kStages);
+  if (warp == 0)
+    for (int k = 0; k < issued; ++k) issue(k);
   pdl_launch_dependents();
 
-  constexpr int LPB = D / 8;           // lanes per block in the dot phase
-  constexpr int BPP = 32 / LPB;        // blocks per warp per pass
-  constexpr int PASSES = kTile / (kWarps * BPP);
-  constexpr int LPH = LPB / G;         // lanes per head after the transpose-reduce
-  constexpr int NC4 = D / 4;
-  constexpr int NJS = kThreads / NC4;  // block subsets of the accumulation phase
+  constexpr int LPB = D / 8;            // lanes per block in the dot phase
+  constexpr int BPP = 32 / LPB;         // blocks per warp per pass
+  constexpr int PASSES = kBlocksPerWarp / BPP;
+  constexpr int LPH = LPB / G;          // lanes per head after the transpose-reduce
+  constexpr int LR = D / 4;             // lanes per mean-value row (4 channels per lane)
+  constexpr int RS = 32 / LR;           // mean-value rows per warp step
+  constexpr int NSL = kWarps * BPP;     // head lanes per head in the CTA
   const int li = lane % LPB, bsub = lane / LPB;
   const bool head_lane = (li % LPH) == 0;
   const int my_h = li / LPH;
-  const int c4 = tid % NC4, js = tid / NC4;
-  // lane-slot index of this head lane among all head lanes of head my_h (for reductions)
-  const int slot = warp * BPP + bsub;  // < kWarps * BPP <= 32
+  const int c4 = lane % LR, rsub = lane / LR;
+  const int slot = warp * BPP + bsub;
 
   float qreg[G][8];
   float acc[G][4];
+  float mref[G];
   float zmax = -CUDART_INF_F, zsum = 0.f, lsum = 0.f;
   int cur = -1;
-  int issued = min(nt, kStages - 1);
 
-  // Writes the partials of the current segment (pair `cur`) and clears the running state.
+  // Merges the 8 warps' partials of the current segment (pair `cur`) in a fixed order.
   auto finish_segment = [&]() {
-    if (head_lane) {
-      red_s[(0 * G + my_h) * 64 + slot] = zmax;
-      red_s[(1 * G + my_h) * 64 + slot] = zsum;
-      red_s[(2 * G + my_h) * 64 + slot] = lsum;
+    if (RS > 1 && compensate) {  // fold the row subsets of each warp (D < 128)
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int o = LR; o < 32; o <<= 1) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], o);
     }
-    if (compensate) {  // fixed order over the block subsets, so results are deterministic
-      for (int w = 0; w < NJS; ++w) {
-        if (js == w) {
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) refw_s[warp * G + h] = mref[h];
+    }
+    if (head_lane) {
+      red_s[(0 * G + my_h) * 32 + slot] = zmax;
+      red_s[(1 * G + my_h) * 32 + slot] = zsum;
+    }
+    for (int i = tid; i < G * D; i += kThreads) comp_s[i] = 0.f;
+    __syncthreads();
+    float M[G], fw[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      M[h] = -CUDART_INF_F;
+      for (int w = 0; w < kWarps; ++w) M[h] = fmaxf(M[h], refw_s[w * G + h]);
+      fw[h] = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - M[h]);
+    }
+    if (head_lane) red_s[(2 * G + my_h) * 32 + slot] = lsum * pick_h<G>(fw, my_h);
+    if (compensate) {
+      for (int w = 0; w < kWarps; ++w) {
+        if (warp == w && rsub == 0) {
 #pragma unroll
           for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) comp_s[h * D + c4 * 4 + e] += acc[h][e];
+            for (int e = 0; e < 4; ++e) comp_s[h * D + c4 * 4 + e] += fw[h] * acc[h][e];
         }
         __syncthreads();
       }
+    } else {
+      __syncthreads();
     }
-    __syncthreads();
     const int k = blockIdx.x - static_cast<int>(((static_cast<long long>(cur) * TP + 1) * p.nctas - 1) / F);
     const size_t rec = static_cast<size_t>(cur) * p.slots + k;
-    constexpr int NSL = kWarps * BPP;
     if (tid < G) {
       float zm = -CUDART_INF_F, zs = 0.f, ls = 0.f;
       for (int s = 0; s < NSL; ++s) {
-        lse_merge(zm, zs, red_s[(0 * G + tid) * 64 + s], red_s[(1 * G + tid) * 64 + s]);
-        ls += red_s[(2 * G + tid) * 64 + s];
+        lse_merge(zm, zs, red_s[(0 * G + tid) * 32 + s], red_s[(1 * G + tid) * 32 + s]);
+        ls += red_s[(2 * G + tid) * 32 + s];
       }
       p.zpart[(rec * G + tid) * 2] = zm;
       p.zpart[(rec * G + tid) * 2 + 1] = zs;
       if (compensate) {
-        p.comp[(rec * G + tid) * (D + 2)] = mref_s[tid];
+        p.comp[(rec * G + tid) * (D + 2)] = pick_h<G>(M, tid);
         p.comp[(rec * G + tid) * (D + 2) + 1] = ls;
       }
     }
@@ -199,13 +232,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   // Loads the query heads of pair `pr` and resets the running state.
   auto start_segment = [&](int pr) {
     const TQ* qp = static_cast<const TQ*>(p.q) + static_cast<size_t>(pr) * G * D;
-    for (int i = tid; i < G * D; i += kThreads) {
-      q_s[i] = to_float(qp[i]);
-      comp_s[i] = 0.f;
-    }
-    if (tid < 8) mref_s[tid] = -CUDART_INF_F;
-    if (tid < 24) tmax_s[tid] = ord_float(-CUDART_INF_F);
-    if (tid < 3) flag_s[tid] = 0;
+    for (int i = tid; i < G * D; i += kThreads) q_s[i] = to_float(qp[i]);
     __syncthreads();
     const int gsz = D / r;
     for (int i = tid; i < G * r; i += kThreads) {
@@ -223,57 +250,63 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       for (int e = 0; e < 4; ++e) {
         qreg[h][e] = q_s[h * D + li * 4 + e];
         qreg[h][4 + e] = q_s[h * D + D / 2 + li * 4 + e];
+        acc[h][e] = 0.f;
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+      mref[h] = -CUDART_INF_F;
     }
     zmax = -CUDART_INF_F;
     zsum = lsum = 0.f;
     __syncthreads();
   };
 
+  // `ok` goes false (for this warp) once a wait gives up; the warp then stops waiting and
+  // computing but keeps the loop's structure, so every CTA barrier stays matched.
   bool ok = true;
-  int waited = nt;
+  int first_unwaited = nt;
 #pragma unroll 1
   for (int k = 0; k < nt; ++k) {
     const int f = f0 + k;
-    const int pr = tile_pair(f);
-    if (pr != cur) {
+    const int pr = f / TP;
+    if (pr != cur) {  // every warp reaches this at the same tile
+      __syncthreads();
       if (cur >= 0) finish_segment();
       start_segment(pr);
       cur = pr;
     }
-    const int jt0 = (f % TP) * kTile;
-    const int tn = min(kTile, p.Nb - jt0);
     const int st = k % kStages;
+    // warp 0 refills the stage of tile k + kStages - 1 once every warp has released tile k - 1
+    if (warp == 0 && k >= 1 && k + kStages - 1 < nt) {
+      const int kk = k + kStages - 1;
+      bool freed = ok && mbar_wait(&empty[kk % kStages], ((kk / kStages) - 1) & 1, p.status);
+      freed = __all_sync(0xffffffffu, freed);
+      if (freed) {
+        issue(kk);
+        ++issued;
+      } else {
+        ok = false;
+      }
+    }
+    bool got = ok && mbar_wait(&full[st], (k / kStages) & 1, p.status);
+    got = __all_sync(0xffffffffu, got);
+    if (!got && ok) {
+      ok = false;
+      first_unwaited = k;
+    }
+    const int jt0 = (f % TP) * kTile;
+    const int tn = ok ? min(kTile, p.Nb - jt0) : 0;
     const unsigned char* sb = sm + L.stage0 + L.stage_bytes * st;
     const float* mu_t = reinterpret_cast<const float*>(sb + L.off_mu);
     const float* nu_t = reinterpret_cast<const float*>(sb + L.off_nu);
     const float* var_t = reinterpret_cast<const float*>(sb + L.off_var);
     const int* cnt_t = reinterpret_cast<const int*>(sb + L.off_cnt);
-    // weights: double buffer (written in phase 1 of tile k, read after its barrier). Tile max and
-    // the reference flag: 3-deep ring; thread 0 clears tile k+1's entry here, which lies after
-    // the barrier that ends tile k-2's readers and before the barrier that starts tile k+1.
-    float* ws_b = ws_s + (k & 1) * kTile * G;
-    const int buf = k % 3;
-    if (tid == 0) {
-      const int nb3 = (k + 1) % 3;
-#pragma unroll
-      for (int h = 0; h < 8; ++h) tmax_s[nb3 * 8 + h] = ord_float(-CUDART_INF_F);
-      flag_s[nb3] = 0;
-    }
-    const bool got = mbar_wait(&mbar[st], (k / kStages) & 1, p.status);
 
-    // ---- (1) dots, scalars, log scores, running Zhat and compensation sums
-    float xs[PASSES], wv[PASSES];
-    const float mref = compensate ? mref_s[my_h] : 0.f;
-    const float lprev = lsum;
+    // ---- (1) dots of this warp's blocks with the G heads
+    float v[PASSES][G];
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) {
-      const int jt = pass * kWarps * BPP + warp * BPP + bsub;
+      const int jt = warp * kBlocksPerWarp + pass * BPP + bsub;
       const float4 a = reinterpret_cast<const float4*>(mu_t + jt * D)[li];
       const float4 b = reinterpret_cast<const float4*>(mu_t + jt * D + D / 2)[li];
-      float v[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float s = qreg[h][0] * a.x;
@@ -284,99 +317,101 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
         s = fmaf(qreg[h][5], b.y, s);
         s = fmaf(qreg[h][6], b.z, s);
         s = fmaf(qreg[h][7], b.w, s);
-        v[h] = s;
+        v[pass][h] = s;
       }
-      TransposeReduce<G, LPB / 2>::run(v, li);
+    }
+#pragma unroll
+    for (int pass = 0; pass < PASSES; ++pass) TransposeReduce<G, LPB / 2>::run(v[pass], li);
+
+    // ---- (2) per (block, head) scalars on the head lanes
+    float xs[PASSES];
+    bool need = false;
+    const float mh0 = pick_h<G>(mref, my_h);
+#pragma unroll
+    for (int pass = 0; pass < PASSES; ++pass) {
+      const int jt = warp * kBlocksPerWarp + pass * BPP + bsub;
       xs[pass] = -CUDART_INF_F;
-      wv[pass] = 0.f;
       if (head_lane && jt < tn) {
         const int n = cnt_t[jt];
         float vh = 0.f;
         for (int g = 0; g < r; ++g) vh = fmaf(qn_s[my_h * r + g], var_t[jt * r + g], vh);
-        const float lbar = p.scale * v[0];
-        float uu;
+        const float lbar = p.scale * v[pass][0];
+        const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jt;
+        float uu, x = -CUDART_INF_F;
         if (n > 0) {
-          const float x = lbar + logn_s[min(n, 16)];
+          x = lbar + logn_s[min(n, 16)];
           const float lm = x + __logf(1.f + 0.5f * vh);
           uu = (p.mode == COMPKV_MODE_COMPKV) ? lm + __logf(0.5f * vh) : lm;
-          xs[pass] = x;
           if (lm > zmax) {
             zsum = zsum * __expf(zmax - lm) + 1.f;
             zmax = lm;
           } else {
             zsum += __expf(lm - zmax);
           }
-          if (compensate) {
-            atomicMax(&tmax_s[buf * 8 + my_h], ord_float(x));
-            if (x > mref + kRefSlack) flag_s[buf] = 1;
-            else wv[pass] = __expf(x - mref);
-          }
+          need = need || (x > mh0 + kRefSlack);
         } else {
           uu = __int_as_float(0x7fffffff);  // NaN marks an empty block
         }
-        p.u[((static_cast<size_t>(pr) * p.Nb) + jt0 + jt) * G + my_h] = uu;
+        xs[pass] = x;
+        p.u[row * G + my_h] = uu;
+        p.xrec[row * XS + my_h] = x;
+        if (my_h == 0) p.xrec[row * XS + G] = __int_as_float(n);
       }
-      if (compensate && head_lane) {
-        ws_b[jt * G + my_h] = wv[pass];
-        lsum += wv[pass];
-      }
-    }
-    ok = __syncthreads_and(got) != 0;
-    if (!ok) {
-      waited = k;
-      break;
-    }
-    if (k + kStages - 1 < nt) {
-      issue(k + kStages - 1);
-      ++issued;
     }
     if (compensate) {
-      if (flag_s[buf]) {  // rare: move the reference of the heads that need it and rescale
-        if (tid < G) {
-          const float old = mref_s[tid];
-          const float tm = unord_float(tmax_s[buf * 8 + tid]);
-          const float nm = (tm > old + kRefSlack) ? tm : old;
-          sc_s[tid] = (old == -CUDART_INF_F) ? 0.f : __expf(old - nm);
-          mref_s[tid] = nm;
-        }
-        __syncthreads();
-        const float nref = mref_s[my_h];
-        lsum = lprev * sc_s[my_h];
-#pragma unroll
-        for (int pass = 0; pass < PASSES; ++pass) {
-          const int jt = pass * kWarps * BPP + warp * BPP + bsub;
-          const float w = (xs[pass] == -CUDART_INF_F) ? 0.f : __expf(xs[pass] - nref);
-          if (head_lane) {
-            ws_b[jt * G + my_h] = w;
-            lsum += w;
-          }
-        }
+      if (__any_sync(0xffffffffu, need)) {  // rare: move this warp's reference up
+        float sc_mine = 1.f;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float sc = sc_s[h];
+          float m = -CUDART_INF_F;
+#pragma unroll
+          for (int pass = 0; pass < PASSES; ++pass) m = fmaxf(m, (head_lane && my_h == h) ? xs[pass] : -CUDART_INF_F);
+          const float tm = warp_max(m);
+          const float nm = (tm > mref[h] + kRefSlack) ? tm : mref[h];
+          const float sc = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - nm);
           acc[h][0] *= sc; acc[h][1] *= sc; acc[h][2] *= sc; acc[h][3] *= sc;
+          if (my_h == h) sc_mine = sc;
+          mref[h] = nm;
         }
-        __syncthreads();
+        lsum *= sc_mine;
       }
-      // ---- (2) acc_h += w_{j,h} nu_j: 4 channels x G heads per thread
-      for (int jt = js; jt < tn; jt += NJS) {
-        const float4 nv = reinterpret_cast<const float4*>(nu_t + jt * D)[c4];
+      const float mh = pick_h<G>(mref, my_h);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float w = ws_b[jt * G + h];
-          acc[h][0] = fmaf(w, nv.x, acc[h][0]);
-          acc[h][1] = fmaf(w, nv.y, acc[h][1]);
-          acc[h][2] = fmaf(w, nv.z, acc[h][2]);
-          acc[h][3] = fmaf(w, nv.w, acc[h][3]);
+      for (int pass = 0; pass < PASSES; ++pass) {
+        const float w = (xs[pass] == -CUDART_INF_F) ? 0.f : __expf(xs[pass] - mh);
+        if (head_lane) {
+          wsw[(pass * BPP + bsub) * G + my_h] = w;
+          lsum += w;
+        }
+      }
+      __syncwarp();
+      // ---- (3) acc_h += w_{j,h} nu_j over this warp's blocks: 4 channels x G heads per lane
+#pragma unroll
+      for (int b0 = 0; b0 < kBlocksPerWarp; b0 += RS) {
+        const int bl = b0 + rsub;
+        const int jt = warp * kBlocksPerWarp + bl;
+        if (jt < tn) {
+          const float4 nv = reinterpret_cast<const float4*>(nu_t + jt * D)[c4];
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float w = wsw[bl * G + h];
+            acc[h][0] = fmaf(w, nv.x, acc[h][0]);
+            acc[h][1] = fmaf(w, nv.y, acc[h][1]);
+            acc[h][2] = fmaf(w, nv.z, acc[h][2]);
+            acc[h][3] = fmaf(w, nv.w, acc[h][3]);
+          }
         }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
   }
-  if (!ok) {
-    for (int k = waited; k < issued; ++k) mbar_wait(&mbar[k % kStages], (k / kStages) & 1, nullptr);
-  } else if (cur >= 0) {
-    finish_segment();
+  if (!ok && warp == 0) {
+    // a wait gave up (status recorded): wait, bounded, for the copies warp 0 issued
+    for (int k = first_unwaited; k < issued; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, nullptr);
   }
+  __syncthreads();
+  if (cur >= 0) finish_segment();
 }
 
 template <typename TQ, int D, int G>
@@ -403,7 +438,7 @@ const void* pick(bool bf16, int D, int G) {
 
 struct Grid {
   const void* kern = nullptr;
-  int dev = -1, D = 0, G = 0, r = 0;
+  int dev = -1, r = 0;
   int ctas_per_sm = 0, sms = 0;
   size_t smem = 0;
 };
@@ -423,8 +458,6 @@ cudaError_t grid_for(const void* kern, int D, int G, int r, Grid* out) {
   Grid g;
   g.kern = kern;
   g.dev = dev;
-  g.D = D;
-  g.G = G;
   g.r = r;
   SLay L;
   L.build(D, G, r);
@@ -440,14 +473,14 @@ cudaError_t grid_for(const void* kern, int D, int G, int r, Grid* out) {
   return cudaSuccess;
 }
 
-}  // namespace
-
 int stream_ctas(int total_tiles, int sms, int ctas_per_sm) {
   int n = sms * (ctas_per_sm < 2 ? ctas_per_sm : 2);
   if (n > kStreamMaxCtas) n = kStreamMaxCtas;
   if (n > total_tiles) n = total_tiles;
   return n < 1 ? 1 : n;
 }
+
+}  // namespace
 
 cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   const void* kern = pick(a.bf16, a.D, a.G);
@@ -470,6 +503,7 @@ cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   p.mean_v = a.mean_v;
   p.count = a.count;
   p.u = a.u;
+  p.xrec = a.xrec;
   p.zpart = a.zpart;
   p.comp = a.comp_seg;
   p.status = a.status;

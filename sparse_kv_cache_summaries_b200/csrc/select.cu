@@ -31,7 +31,7 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast
 
 struct SelLay {
   int chunk, cand_cap, gcap, slots, G;
-  size_t keys, cand_key, cand_idx, gkey, gidx, hist, bc, scan, misc, zm, zs, fac, total;
+  size_t keys, cand_key, cand_idx, gkey, gidx, hist, bc, scan, misc, zm, zs, fac, cl, mrg, total;
   __host__ __device__ void build(int chunk_, int Kb, int C, int slots_, int G_) {
     chunk = chunk_;
     slots = slots_;
@@ -51,6 +51,8 @@ struct SelLay {
     zm = o;       o = a16(o + sizeof(float) * slots * G);
     zs = o;       o = a16(o + sizeof(float) * slots * G);
     fac = o;      o = a16(o + sizeof(float) * slots * G);
+    cl = o;       o = a16(o + sizeof(float) * slots * G);
+    mrg = o;      o = a16(o + sizeof(float) * kThreads);
     total = o;
   }
 };
@@ -102,14 +104,19 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
   const int nseg = stream_cta_of_tile(f_first + p.tiles_per_pair - 1, p.nctas_stream, p.total_tiles) - c_first + 1;
 
   pdl_wait();  // the streaming kernel's outputs are visible from here on
+  pdl_launch_dependents();
 
-  // ---- log Zhat per head from the segment partials (and the compensation maxima)
+  // ---- log Zhat per head from the segment partials, and the compensation maxima and sums
+  float* cl_s = reinterpret_cast<float*>(sm + L.cl);
   const float* zp = p.zpart + static_cast<size_t>(pr) * p.slots * G * 2;
   const float* cs = p.comp_seg + static_cast<size_t>(pr) * p.slots * G * (D + 2);
   for (int t = tid; t < nseg * G; t += kThreads) {
     zm_s[t] = zp[2 * t];
     zs_s[t] = zp[2 * t + 1];
-    if (compensate) fac_s[t] = cs[static_cast<size_t>(t) * (D + 2)];
+    if (compensate) {
+      fac_s[t] = cs[static_cast<size_t>(t) * (D + 2)];
+      cl_s[t] = cs[static_cast<size_t>(t) * (D + 2) + 1];
+    }
   }
   __syncthreads();
   if (warp < G) {
@@ -123,7 +130,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
       lse_merge(m, s, m2, s2);
     }
     if (lane == 0) logz[h] = (m == -CUDART_INF_F) ? -CUDART_INF_F : m + logf(s);
-    if (compensate) {  // common max of the compensation partials and their factors
+    if (compensate) {  // common max of the compensation partials, their factors and the sum l
       float M = -CUDART_INF_F;
       for (int t = lane; t < nseg; t += 32) M = fmaxf(M, fac_s[t * G + h]);
       M = warp_max(M);
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
         const float mt = fac_s[t * G + h];
         const float f = (mt == -CUDART_INF_F) ? 0.f : __expf(mt - M);
         fac_s[t * G + h] = f;
-        l = fmaf(f, cs[(static_cast<size_t>(t) * G + h) * (D + 2) + 1], l);
+        l = fmaf(f, cl_s[t * G + h], l);
       }
       l = warp_sum(l);
       if (rank == 0 && lane == 0) {
@@ -183,19 +190,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
     if (tid == 0) misc[0] = ncand;
   }
 
-  // ---- merge this rank's slice of the compensation partials
-  if (compensate) {
-    const int E = G * D;
-    const int per = (E + C - 1) / C;
-    const int e0 = rank * per, e1 = min(E, e0 + per);
-    for (int e = e0 + tid; e < e1; e += kThreads) {
-      const int h = e / D, c = e % D;
-      float a = 0.f;
-#pragma unroll 4
-      for (int t = 0; t < nseg; ++t) a = fmaf(fac_s[t * G + h], cs[(static_cast<size_t>(t) * G + h) * (D + 2) + 2 + c], a);
-      p.comp[(static_cast<size_t>(pr) * G + h) * (D + 2) + 2 + c] = a;
-    }
-  }
   cluster.sync();  // #1: every rank's candidates are visible
 
   if (rank == 0 && Kb > 0) {
@@ -220,8 +214,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
       gidx[i] = *cluster.map_shared_rank(&cand_idx[k], c);
     }
   }
-  cluster.sync();  // #2: no rank reads another rank's shared memory after this
-
   if (rank == 0 && Kb > 0) {
     const int M = misc[1];
     int32_t* sel = p.sel_idx + static_cast<size_t>(pr) * Kb;
@@ -233,7 +225,34 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
       cta_select_ordered(kat, M, cut, scan, [&](int i, int pos) { sel[pos] = gidx[i]; });
     }
   }
-  pdl_launch_dependents();
+  if (compensate && (C == 1 || rank != 0)) {
+    // merge a slice of the compensation partials' channels: lanes along channels (coalesced),
+    // 4 segment groups per slice summed in a fixed order
+    float* mrg = reinterpret_cast<float*>(sm + L.mrg);
+    const int E = G * D, W = (C == 1) ? 1 : C - 1, wr = (C == 1) ? 0 : rank - 1;
+    const int per = (E + W - 1) / W;
+    const int e0 = wr * per, e1 = min(E, e0 + per);
+    const int ei = tid % 64, sg = tid / 64;
+    for (int base = e0; base < e1; base += 64) {
+      const int e = base + ei;
+      float a = 0.f;
+      if (e < e1) {
+        const int h = e / D, c = e % D;
+#pragma unroll 8
+        for (int t = sg; t < nseg; t += 4)
+          a = fmaf(fac_s[t * G + h], cs[(static_cast<size_t>(t) * G + h) * (D + 2) + 2 + c], a);
+      }
+      mrg[sg * 64 + ei] = a;
+      __syncthreads();
+      if (tid < 64 && base + tid < e1) {
+        const int e2 = base + tid;
+        p.comp[(static_cast<size_t>(pr) * G + e2 / D) * (D + 2) + 2 + (e2 % D)] =
+            ((mrg[tid] + mrg[64 + tid]) + mrg[128 + tid]) + mrg[192 + tid];
+      }
+      __syncthreads();
+    }
+  }
+  cluster.sync();  // #2: no rank reads another rank's shared memory after this
 }
 
 template <int G, int D>

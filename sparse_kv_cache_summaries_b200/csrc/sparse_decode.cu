@@ -36,11 +36,10 @@ struct SParams {
   const void* q;
   const void* K;
   const void* V;
-  const float* mean_k;
   const float* mean_v;
-  const int32_t* count;
   const int32_t* sel_idx;
   const float* comp;
+  const float* xrec;
   float* out;
   int32_t* status;
 };
@@ -50,18 +49,20 @@ struct SLayout {
   static constexpr size_t kv_bytes = sizeof(T) * kRows * D;
   static constexpr size_t off_k = 0;
   static constexpr size_t off_v = off_k + kv_bytes;
-  static constexpr size_t off_lg = off_v + kv_bytes;                     // [G][kRows]
+  static constexpr size_t off_nu = off_v + kv_bytes;                     // [kRound][D] fp32
+  static constexpr size_t off_lg = off_nu + sizeof(float) * kRound * D;  // [G][kRows]
   static constexpr size_t off_p = off_lg + sizeof(float) * G * kRows;    // [kRows][G]
   static constexpr size_t off_q = off_p + sizeof(float) * G * kRows;     // [G][D]
   static constexpr size_t off_red = off_q + sizeof(float) * G * D;       // [kSub][G][D]
   static constexpr size_t off_acc = off_red + sizeof(float) * PV<T, D, G>::kSub * G * D;  // [G][D]
-  static constexpr size_t off_ml = off_acc + sizeof(float) * G * D;      // [G][2]
-  static constexpr size_t off_blk = off_ml + sizeof(float) * 2 * 8;      // j, n, slot flags
-  static constexpr size_t off_lbar = off_blk + sizeof(int) * 2 * kRound; // [G][kRound]
-  static constexpr size_t off_pw = off_lbar + sizeof(float) * G * 17;
+  static constexpr size_t off_cp = off_acc + sizeof(float) * G * D;      // [G][D+2] compensation
+  static constexpr size_t off_ml = off_cp + sizeof(float) * G * (D + 2); // [G][2]
+  static constexpr size_t off_blk = off_ml + sizeof(float) * 2 * 8;      // j, n
+  static constexpr size_t off_xr = off_blk + sizeof(int) * 2 * kRound;   // [kRound][G] x
+  static constexpr size_t off_pw = off_xr + sizeof(float) * G * kRound;  // [G][kRound]
   static constexpr size_t off_sc = off_pw + sizeof(float) * G * kRound;  // [G]
-  static constexpr size_t off_fac = off_sc + sizeof(float) * 8;          // [G][17]
-  static constexpr size_t off_mbar = (off_fac + sizeof(float) * G * 17 + 15) & ~size_t(15);
+  static constexpr size_t off_fac = off_sc + sizeof(float) * 8;          // [G][17] x 2
+  static constexpr size_t off_mbar = (off_fac + sizeof(float) * G * 34 + 15) & ~size_t(15);
   static constexpr size_t total = off_mbar + 16;
 };
 
@@ -71,30 +72,34 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
   using RG = RowGeom<T, D>;
   using PVt = PV<T, D, G>;
   constexpr int EPV = RG::kEpv, VEC = PVt::kVec;
+  constexpr int XS = xrec_stride(G);
   extern __shared__ __align__(128) unsigned char sm[];
   T* kbuf = reinterpret_cast<T*>(sm + LY::off_k);
   T* vbuf = reinterpret_cast<T*>(sm + LY::off_v);
+  float* nu_s = reinterpret_cast<float*>(sm + LY::off_nu);
   float* lg = reinterpret_cast<float*>(sm + LY::off_lg);
   float* pT = reinterpret_cast<float*>(sm + LY::off_p);
   float* q_s = reinterpret_cast<float*>(sm + LY::off_q);
   float* red = reinterpret_cast<float*>(sm + LY::off_red);
   float* acc_s = reinterpret_cast<float*>(sm + LY::off_acc);
+  float* cp_s = reinterpret_cast<float*>(sm + LY::off_cp);
   float* ml_s = reinterpret_cast<float*>(sm + LY::off_ml);
   int* blk_j = reinterpret_cast<int*>(sm + LY::off_blk);
   int* blk_n = blk_j + kRound;
-  float* lbar_s = reinterpret_cast<float*>(sm + LY::off_lbar);
+  float* xr_s = reinterpret_cast<float*>(sm + LY::off_xr);
   float* pw_s = reinterpret_cast<float*>(sm + LY::off_pw);
   float* sc_s = reinterpret_cast<float*>(sm + LY::off_sc);
   float* fac_s = reinterpret_cast<float*>(sm + LY::off_fac);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + LY::off_mbar);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int NS = static_cast<int>(cluster_size());
-  const int rank = static_cast<int>(cluster_rank());
+  cg::cluster_group cluster = cg::this_cluster();
+  const int NS = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
   const int bk = blockIdx.x / NS;
   const bool compensate = p.mode != COMPKV_MODE_MASS;
 
-  // ---- prologue (inputs written before the score kernel started)
+  // ---- prologue: inputs written before the select kernel started
   if (tid == 0) {
     mbar_init(mbar, 1);
     mbar_init_fence();
@@ -115,68 +120,63 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
     for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
   float m_run = -CUDART_INF_F, l_run = 0.f;  // warp h's running state for head h
 
-  pdl_wait();  // selection and compensation partials of the score kernel are now visible
+  pdl_wait();  // selection, records and compensation partial are visible from here on
 
+  if (rank == 0 && compensate) {  // prefetch the compensation partial for the merge
+    const float* cp = p.comp + static_cast<size_t>(bk) * G * (D + 2);
+    for (int i = tid; i < G * (D + 2); i += kThreads) cp_s[i] = cp[i];
+  }
   const T* Kbase = static_cast<const T*>(p.K) + static_cast<size_t>(bk) * p.T * D;
   const T* Vbase = static_cast<const T*>(p.V) + static_cast<size_t>(bk) * p.T * D;
+  const float* NUbase = p.mean_v + static_cast<size_t>(bk) * p.Nb * D;
+  const float* XRbase = p.xrec + static_cast<size_t>(bk) * p.Nb * XS;
   const int s0 = rank * p.bpc;
   const int s1 = min(p.Kb, s0 + p.bpc);
   uint32_t phase = 0;
-  bool ok = true;
-  (void)ok;
 #pragma unroll 1
   for (int rs0 = s0; rs0 < s1; rs0 += kRound) {
     const int nr = min(kRound, s1 - rs0);
     if (tid < kRound) {
-      int j = -1, n = 0;
+      int j = -1;
       if (tid < nr) {
         j = p.sel_idx[static_cast<size_t>(bk) * p.Kb + rs0 + tid];
-        if (j >= 0 && j < p.Nb) n = p.count[static_cast<size_t>(bk) * p.Nb + j];
-        n = max(0, min(n, kBlockTokens));
         if (j < 0 || j >= p.Nb) j = -1;
       }
       blk_j[tid] = j;
-      blk_n[tid] = n;
     }
     __syncthreads();
+    // K and V rows up to the cache capacity (the block's token count arrives with its record)
     if (tid == 0) {
       uint32_t bytes = 0;
-      for (int s = 0; s < nr; ++s) bytes += 2u * blk_n[s] * D * sizeof(T);
+      for (int s = 0; s < nr; ++s) {
+        const int j = blk_j[s];
+        if (j < 0) continue;
+        const int rows = min(kBlockTokens, p.T - j * kBlockTokens);
+        bytes += 2u * rows * D * sizeof(T) + (compensate ? D * sizeof(float) : 0u);
+      }
       mbar_arrive_expect_tx(mbar, bytes);
       for (int s = 0; s < nr; ++s) {
-        const int n = blk_n[s];
-        if (n == 0) continue;
-        const size_t off = static_cast<size_t>(blk_j[s]) * kBlockTokens * D;
-        bulk_g2s(kbuf + s * kBlockTokens * D, Kbase + off, n * D * sizeof(T), mbar);
-        bulk_g2s(vbuf + s * kBlockTokens * D, Vbase + off, n * D * sizeof(T), mbar);
+        const int j = blk_j[s];
+        if (j < 0) continue;
+        const int rows = min(kBlockTokens, p.T - j * kBlockTokens);
+        const size_t off = static_cast<size_t>(j) * kBlockTokens * D;
+        bulk_g2s(kbuf + s * kBlockTokens * D, Kbase + off, rows * D * sizeof(T), mbar);
+        bulk_g2s(vbuf + s * kBlockTokens * D, Vbase + off, rows * D * sizeof(T), mbar);
+        if (compensate) bulk_g2s(nu_s + s * D, NUbase + static_cast<size_t>(j) * D, D * sizeof(float), mbar);
       }
     }
-    // block-mean logits of the selected blocks (for removing their compensation terms)
-    if (compensate) {
-      for (int s = warp; s < nr; s += kWarps) {
-        float v[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) v[h] = 0.f;
-        if (blk_n[s] > 0) {
-          const float* mk = p.mean_k + (static_cast<size_t>(bk) * p.Nb + blk_j[s]) * D;
-          for (int c = lane; c < D; c += 32) {
-            const float x = mk[c];
-#pragma unroll
-            for (int h = 0; h < G; ++h) v[h] = fmaf(q_s[h * D + c], x, v[h]);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) v[h] = warp_sum(v[h]);
-        if (lane < G) {
-          float x = v[0];
-#pragma unroll
-          for (int h = 1; h < G; ++h) x = (lane == h) ? v[h] : x;
-          lbar_s[lane * kRound + s] = p.scale * x;
-        }
-      }
+    // records: x_h and the token count of each selected block
+    if (tid < nr * (G + 1)) {
+      const int s = tid / (G + 1), e = tid % (G + 1);
+      const int j = blk_j[s];
+      const float v = (j >= 0) ? XRbase[static_cast<size_t>(j) * XS + e] : 0.f;
+      if (e < G) xr_s[s * G + e] = (j >= 0) ? v : -CUDART_INF_F;
+      else blk_n[s] = (j >= 0) ? max(0, min(__float_as_int(v), min(kBlockTokens, p.T - j * kBlockTokens))) : 0;
     }
+    if (tid >= nr && tid < kRound) blk_n[tid] = 0;
     const bool got = mbar_wait(mbar, phase, p.status);
-    // rows of a partial block that no copy wrote: zero V (their weight is 0, but 0 * NaN is not)
+    __syncthreads();  // records visible
+    // V rows past a block's token count: zero them (their weight is 0, but 0 * NaN is not)
     for (int s = 0; s < nr; ++s) {
       const int n = blk_n[s];
       if (n < kBlockTokens) {
@@ -185,8 +185,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
       }
     }
     fence_proxy_async();  // the next round's copies may land on these rows
-    ok = __syncthreads_and(got) != 0;
-    if (!ok) {  // uniform: drain (bounded) and stop
+    if (__syncthreads_and(got) == 0) {  // uniform: drain (bounded) and stop
       mbar_wait(mbar, phase, nullptr);
       break;
     }
@@ -199,7 +198,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
       return row < R && (row % kBlockTokens) < blk_n[row / kBlockTokens];
     });
     __syncthreads();
-    // softmax update, warp h for head h
+    // softmax update, warp h for head h; compensation terms of the selected blocks removed
     if (warp < G) {
       const int h = warp;
       float mx = -CUDART_INF_F;
@@ -215,8 +214,9 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
       }
       ls = warp_sum(ls);
       float pw = 0.f;
-      if (compensate && lane < nr && blk_n[lane] > 0) {
-        pw = __expf(lbar_s[h * kRound + lane] + logf(static_cast<float>(blk_n[lane])) - m_new);
+      if (compensate && lane < nr) {
+        const float xj = xr_s[lane * G + h];
+        pw = (xj == -CUDART_INF_F) ? 0.f : __expf(xj - m_new);
       }
       if (lane < kRound) pw_s[h * kRound + lane] = pw;
       const float pws = warp_sum(pw);
@@ -226,7 +226,6 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
       if (lane == 0) sc_s[h] = sc;
     }
     __syncthreads();
-    // P.V and removal of the selected blocks' compensation terms
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float sc = sc_s[h];
@@ -236,11 +235,9 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
     PVt::accumulate(vbuf, pT, R, sub, cv, acc);
     if (compensate && sub == 0) {
       for (int s = 0; s < nr; ++s) {
-        if (blk_n[s] == 0) continue;
-        const float* mv = p.mean_v + (static_cast<size_t>(bk) * p.Nb + blk_j[s]) * D + cv * VEC;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          const float nv = mv[e];
+          const float nv = nu_s[s * D + cv * VEC + e];
 #pragma unroll
           for (int h = 0; h < G; ++h) acc[h][e] = fmaf(-pw_s[h * kRound + s], nv, acc[h][e]);
         }
@@ -264,29 +261,27 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
     for (int k = 0; k < PVt::kSub; ++k) s += red[k * G * D + i];
     acc_s[i] = s;
   }
-  cluster_sync();  // #1: every split's partial is visible
+  cluster.sync();  // #1: every split's partial is visible
 
   if (rank == 0) {
-    cg::cluster_group cluster = cg::this_cluster();
-    const float* cp = p.comp + static_cast<size_t>(bk) * G * (D + 2);
     // per head: common max over the splits and the compensation partial, factors, 1/denominator
     if (tid < G * NS) {
       const int h = tid / NS, s = tid % NS;
       const float* rml = cluster.map_shared_rank(ml_s, s);
       fac_s[h * 17 + s] = rml[2 * h];
-      lbar_s[h * 17 + s] = rml[2 * h + 1];   // reused as scratch for the split denominators
+      fac_s[G * 17 + h * 17 + s] = rml[2 * h + 1];
     }
     __syncthreads();
     if (tid < G) {
       const int h = tid;
-      const float cm = compensate ? cp[h * (D + 2)] : -CUDART_INF_F;
+      const float cm = compensate ? cp_s[h * (D + 2)] : -CUDART_INF_F;
       float M = cm;
       for (int s = 0; s < NS; ++s) M = fmaxf(M, fac_s[h * 17 + s]);
       float den = 0.f;
       if (cm != -CUDART_INF_F) {
         const float f = __expf(cm - M);
         fac_s[h * 17 + 16] = f;
-        den = f * cp[h * (D + 2) + 1];
+        den = f * cp_s[h * (D + 2) + 1];
       } else {
         fac_s[h * 17 + 16] = 0.f;
       }
@@ -294,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
         const float ms = fac_s[h * 17 + s];
         const float f = (ms == -CUDART_INF_F) ? 0.f : __expf(ms - M);
         fac_s[h * 17 + s] = f;
-        den = fmaf(f, lbar_s[h * 17 + s], den);
+        den = fmaf(f, fac_s[G * 17 + h * 17 + s], den);
       }
       sc_s[h] = den > 0.f ? 1.f / den : 0.f;
     }
@@ -305,13 +300,13 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const __grid_co
       float part[16];
 #pragma unroll
       for (int s = 0; s < 16; ++s) part[s] = (s < NS) ? cluster.map_shared_rank(acc_s, s)[i] : 0.f;
-      float a = compensate ? fac_s[h * 17 + 16] * cp[h * (D + 2) + 2 + c] : 0.f;
+      float a = compensate ? fac_s[h * 17 + 16] * cp_s[h * (D + 2) + 2 + c] : 0.f;
 #pragma unroll
       for (int s = 0; s < 16; ++s) a = fmaf(fac_s[h * 17 + s], part[s], a);
       o[i] = a * sc_s[h];
     }
   }
-  cluster_sync();  // #2: rank 0 is done reading the other ranks' shared memory
+  cluster.sync();  // #2: rank 0 is done reading the other ranks' shared memory
 }
 
 template <typename T, int D, int G>
@@ -337,11 +332,10 @@ cudaError_t launch_t(const SparseArgs& a, cudaStream_t st, int bpc, int ns) {
   p.q = a.q;
   p.K = a.K;
   p.V = a.V;
-  p.mean_k = a.mean_k;
   p.mean_v = a.mean_v;
-  p.count = a.count;
   p.sel_idx = a.sel_idx;
   p.comp = a.comp;
+  p.xrec = a.xrec;
   p.out = a.out;
   p.status = a.status;
   cudaLaunchConfig_t cfg = {};
