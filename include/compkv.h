@@ -180,6 +180,36 @@ int compkv_full_decode(const compkv_shape* shape, compkv_dtype dtype, const void
                        float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* Allocation-free decode step. This entry point has no counterpart in the CompKV paper or its  */
+/* review; it is a deployment convenience of this library.                                      */
+
+/* Size of the scratch array inside the library that compkv_decode_step_static uses. */
+#define COMPKV_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* compkv_decode_step for callers that cannot allocate device memory: for example code that runs
+ * inside a host engine which owns every device allocation and only hands out input and output
+ * buffers, or a path where calling cudaMalloc (and the device synchronisation it can cause) is
+ * not allowed. Instead of a caller workspace it uses a scratch array of
+ * COMPKV_STATIC_SCRATCH_BYTES compiled into the library as static device memory; every GPU that
+ * loads the library keeps that array until the process exits. The call itself allocates nothing:
+ * no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - Shapes whose compkv_workspace_bytes(shape, budget_tokens) exceeds
+ *     COMPKV_STATIC_SCRATCH_BYTES are rejected with COMPKV_ERR_WORKSPACE_TOO_SMALL before any
+ *     launch (the 128K-context, 8-kv-head layer needs about 4 MB).
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and keeps it; make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the previous call's contents. Nothing in it has
+ *     to start at zero (each call overwrites what it reads); its device status word is not
+ *     reported by this entry point. Calls that can overlap on the GPU (other streams, other host
+ *     threads) race on the array: the caller must serialise them.
+ * Arguments and outputs are those of compkv_decode_step without workspace and workspace_bytes. */
+int compkv_decode_step_static(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
+                              const void* q, const void* K, const void* V, const float* mean_k,
+                              const float* var_g, const float* mean_v, const int32_t* count,
+                              int32_t budget_tokens, float softmax_scale, int32_t* sel_idx,
+                              float* scores, float* out, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* Diagnostics                                                                                  */
 
 /* Copies the workspace status word (COMPKV_DEVERR_* bits, 0 = clean) to *status (host) and

@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
             "compkv_decode_step": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
                                                   P, P, I32, F, P, P, P, P, SZ, P]),
             "compkv_full_decode": (ctypes.c_int, [SP, ctypes.c_int, P, P, P, P, F, P, P, SZ, P]),
+            "compkv_decode_step_static": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P,
+                                                         P, P, P, P, I32, F, P, P, P, P]),
             "compkv_read_device_status": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
             "compkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "compkv_last_cuda_error": (ctypes.c_char_p, []),
@@ -222,6 +224,20 @@ def decode_step(shape: LayerShape, q: torch.Tensor, K: torch.Tensor, V: torch.Te
                                  _p(summ.count), budget_tokens, softmax_scale, _p(sel_idx),
                                  _p(scores), _p(out), _p(workspace), workspace.numel(),
                                  _stream(stream)), "decode_step")
+    return out
+
+
+def decode_step_static(shape: LayerShape, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                       summ: Summaries, budget_tokens: int, sel_idx: torch.Tensor,
+                       out: torch.Tensor, mode: str = "compkv", scores: torch.Tensor | None = None,
+                       softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+    """decode_step without a workspace: the library's own static device scratch is used (for
+    callers that cannot allocate device memory; see compkv_decode_step_static)."""
+    _ok(lib().compkv_decode_step_static(ctypes.byref(shape.c()), _dt(q), MODES[mode], _p(q),
+                                        _p(K), _p(V), _p(summ.mean_k), _p(summ.var_g),
+                                        _p(summ.mean_v), _p(summ.count), budget_tokens,
+                                        softmax_scale, _p(sel_idx), _p(scores), _p(out),
+                                        _stream(stream)), "decode_step_static")
     return out
 
 
