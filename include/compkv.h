@@ -142,6 +142,18 @@ int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
                         float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* a1, first pass alone: the streaming pass of compkv_score_select over every block's summaries,
+ * without the selection. It leaves in the workspace each block's per-head log score and mean
+ * logit record and the per-segment partials of Zhat and of the compensation sum; nothing else is
+ * written. Exposed so that the pass that reads all the summaries (the bandwidth-bound part of the
+ * step) can be timed on its own; a following compkv_score_select recomputes everything it needs.
+ * Arguments as for compkv_score_select.                                                       */
+int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
+                        const void* q, const float* mean_k, const float* var_g,
+                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        float softmax_scale, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* a3. Exact attention over the selected blocks plus Mean compensation, in one softmax.
  * CompKV abstract ("computing exact attention over a selected subset", compensation of "the
  * omitted attention tail") and review, Summary ("omitted blocks contribute their block-mean
@@ -161,9 +173,10 @@ int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_m
                          int32_t budget_tokens, float softmax_scale, float* out, void* workspace,
                          size_t workspace_bytes, void* stream);
 
-/* One whole decode step: compkv_score_select followed by compkv_sparse_decode (the second kernel
- * is launched with programmatic dependent launch so its prologue overlaps the first's tail).
- * Arguments as above. */
+/* One whole decode step: the result of compkv_score_select followed by compkv_sparse_decode, in
+ * two kernels: the streaming score pass, then one kernel that selects and attends (launched with
+ * programmatic dependent launch so its prologue overlaps the first's tail; the selection is kept
+ * on chip and also written to sel_idx). Arguments as above. */
 int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
                        const void* q, const void* K, const void* V, const float* mean_k,
                        const float* var_g, const float* mean_v, const int32_t* count,

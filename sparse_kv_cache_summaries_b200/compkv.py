@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
             "compkv_build_summaries": (ctypes.c_int, [SP, ctypes.c_int, P, P, P, P, P, P, P, P]),
             "compkv_score_select": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
                                                    I32, F, P, P, P, SZ, P]),
+            "compkv_score_stream": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
+                                                   I32, F, P, SZ, P]),
             "compkv_sparse_decode": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P,
                                                     P, P, P, I32, F, P, P, SZ, P]),
             "compkv_decode_step": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
@@ -201,6 +203,16 @@ def score_select(shape: LayerShape, q: torch.Tensor, summ: Summaries, budget_tok
                                   _p(scores), _p(workspace), workspace.numel(), _stream(stream)),
         "score_select")
     return sel_idx
+
+
+def score_stream(shape: LayerShape, q: torch.Tensor, summ: Summaries, budget_tokens: int,
+                 workspace: torch.Tensor, mode: str = "compkv", softmax_scale: float = 0.0,
+                 stream=None) -> None:
+    """The streaming pass of score_select alone (its outputs stay in the workspace)."""
+    _ok(lib().compkv_score_stream(ctypes.byref(shape.c()), _dt(q), MODES[mode], _p(q),
+                                  _p(summ.mean_k), _p(summ.var_g), _p(summ.mean_v),
+                                  _p(summ.count), budget_tokens, softmax_scale, _p(workspace),
+                                  workspace.numel(), _stream(stream)), "score_stream")
 
 
 def sparse_decode(shape: LayerShape, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,

@@ -146,16 +146,22 @@ int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const 
   return cuda_status(compkv::launch_build_summaries(a, static_cast<cudaStream_t>(stream)));
 }
 
+enum class Upto { kStream, kSelect, kAttend };
+
+// Streaming score kernel, then (unless `upto` is kStream) the select kernel, or with kAttend the
+// select-and-attend kernel, launched with programmatic dependent launch.
 static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
                              const void* q, const float* mean_k, const float* var_g,
                              const float* mean_v, const int32_t* count, int32_t budget_tokens,
                              float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+                             size_t workspace_bytes, void* stream, Upto upto, const void* K,
+                             const void* V, float* out) {
   Common c;
   int st = check_step_args(shape, dtype, mode, budget_tokens, workspace, workspace_bytes, &c);
   if (st) return st;
   const bool comp = mode != COMPKV_MODE_MASS;
-  if (!q || !mean_k || !var_g || !count || (comp && !mean_v) || (c.Kb > 0 && !sel_idx))
+  if (!q || !mean_k || !var_g || !count || (comp && !mean_v) ||
+      (upto != Upto::kStream && c.Kb > 0 && !sel_idx))
     return COMPKV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(mean_k) || (comp && !aligned16(mean_v)) || !aligned4(var_g) ||
       !aligned4(count) || (sel_idx && !aligned4(sel_idx)) || (scores && !aligned4(scores)))
@@ -186,30 +192,63 @@ static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, comp
   a.nctas_out = &nctas;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int rc = cuda_status(compkv::launch_score_stream(a, cs));
-  if (rc) return rc;
-  compkv::SelectArgs b;
+  if (rc || upto == Upto::kStream) return rc;
+  compkv::FusedArgs b;
+  b.bf16 = a.bf16;
   b.mode = mode;
+  b.do_select = true;
+  b.do_attend = upto == Upto::kAttend;
   b.pairs = pairs;
   b.G = c.G;
   b.D = shape->head_dim;
+  b.T = shape->ctx_len;
   b.Nb = c.Nb;
   b.Kb = c.Kb;
   b.slots = W.slots;
   b.nctas_stream = nctas;
+  b.scale = a.scale;
+  b.q = q;
+  b.K = K;
+  b.V = V;
+  b.mean_v = mean_v;
   b.u = a.u;
+  b.xrec = a.xrec;
   b.zpart = a.zpart;
   b.comp_seg = a.comp_seg;
   b.comp = ws_at(workspace, W.comp);
   b.sel_idx = sel_idx;
   b.scores = scores;
-  return cuda_status(compkv::launch_select(b, cs));
+  b.out = out;
+  b.status = a.status;
+  b.pdl = true;
+  return cuda_status(compkv::launch_decode_fused(b, cs));
 }
 
-static int sparse_decode_impl(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                              const void* q, const void* K, const void* V, const float* mean_k,
-                              const float* mean_v, const int32_t* count, const int32_t* sel_idx,
-                              int32_t budget_tokens, float softmax_scale, float* out,
-                              void* workspace, size_t workspace_bytes, void* stream, bool pdl) {
+int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
+                        const void* q, const float* mean_k, const float* var_g,
+                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
+                           softmax_scale, sel_idx, scores, workspace, workspace_bytes, stream,
+                           Upto::kSelect, nullptr, nullptr, nullptr);
+}
+
+int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
+                        const void* q, const float* mean_k, const float* var_g,
+                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        float softmax_scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
+                           softmax_scale, nullptr, nullptr, workspace, workspace_bytes, stream,
+                           Upto::kStream, nullptr, nullptr, nullptr);
+}
+
+int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
+                         const void* q, const void* K, const void* V, const float* mean_k,
+                         const float* mean_v, const int32_t* count, const int32_t* sel_idx,
+                         int32_t budget_tokens, float softmax_scale, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
   Common c;
   int st = check_step_args(shape, dtype, mode, budget_tokens, workspace, workspace_bytes, &c);
   if (st) return st;
@@ -219,49 +258,36 @@ static int sparse_decode_impl(const compkv_shape* shape, compkv_dtype dtype, com
   if (!aligned16(q) || !aligned16(K) || !aligned16(V) || (comp && (!aligned16(mean_k) || !aligned16(mean_v))) ||
       !aligned4(count) || (sel_idx && !aligned4(sel_idx)) || !aligned4(out))
     return COMPKV_ERR_BAD_ALIGNMENT;
-  compkv::SparseArgs a;
-  a.bf16 = dtype == COMPKV_BF16;
-  a.mode = mode;
-  a.B = shape->batch;
-  a.Hkv = shape->n_kv_heads;
-  a.G = c.G;
-  a.D = shape->head_dim;
-  a.T = shape->ctx_len;
-  a.Nb = c.Nb;
-  a.Kb = c.Kb;
-  a.scale = scale_of(shape, softmax_scale);
-  a.q = q;
-  a.K = K;
-  a.V = V;
-  a.mean_k = mean_k;
-  a.mean_v = mean_v;
-  a.count = count;
-  a.sel_idx = sel_idx;
-  a.comp = ws_at(workspace, step_ws(shape).comp);
-  a.xrec = ws_at(workspace, step_ws(shape).xrec);
-  a.out = out;
-  a.status = status_word(workspace);
-  a.pdl = pdl;
-  return cuda_status(compkv::launch_sparse_decode(a, static_cast<cudaStream_t>(stream)));
-}
-
-int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                        const void* q, const float* mean_k, const float* var_g,
-                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
-                        float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
-                        size_t workspace_bytes, void* stream) {
-  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
-                           softmax_scale, sel_idx, scores, workspace, workspace_bytes, stream);
-}
-
-int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                         const void* q, const void* K, const void* V, const float* mean_k,
-                         const float* mean_v, const int32_t* count, const int32_t* sel_idx,
-                         int32_t budget_tokens, float softmax_scale, float* out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
-  return sparse_decode_impl(shape, dtype, mode, q, K, V, mean_k, mean_v, count, sel_idx,
-                            budget_tokens, softmax_scale, out, workspace, workspace_bytes, stream,
-                            false);
+  const compkv::StepWorkspace W = step_ws(shape);
+  compkv::FusedArgs b;
+  b.bf16 = dtype == COMPKV_BF16;
+  b.mode = mode;
+  b.do_select = false;
+  b.do_attend = true;
+  b.pairs = shape->batch * shape->n_kv_heads;
+  b.G = c.G;
+  b.D = shape->head_dim;
+  b.T = shape->ctx_len;
+  b.Nb = c.Nb;
+  b.Kb = c.Kb;
+  b.slots = W.slots;
+  b.nctas_stream = 0;
+  b.scale = scale_of(shape, softmax_scale);
+  b.q = q;
+  b.K = K;
+  b.V = V;
+  b.mean_v = mean_v;
+  b.u = nullptr;
+  b.xrec = ws_at(workspace, W.xrec);
+  b.zpart = nullptr;
+  b.comp_seg = nullptr;
+  b.comp = ws_at(workspace, W.comp);
+  b.sel_idx = const_cast<int32_t*>(sel_idx);  // read only when do_select is false
+  b.scores = nullptr;
+  b.out = out;
+  b.status = status_word(workspace);
+  b.pdl = false;
+  return cuda_status(compkv::launch_decode_fused(b, static_cast<cudaStream_t>(stream)));
 }
 
 int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
@@ -270,18 +296,11 @@ int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mod
                        int32_t budget_tokens, float softmax_scale, int32_t* sel_idx,
                        float* scores, float* out, void* workspace, size_t workspace_bytes,
                        void* stream) {
-  // validate everything the second call needs before launching the first
-  Common c;
-  int st = check_step_args(shape, dtype, mode, budget_tokens, workspace, workspace_bytes, &c);
-  if (st) return st;
   if (!K || !V || !out) return COMPKV_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(V) || !aligned4(out)) return COMPKV_ERR_BAD_ALIGNMENT;
-  st = score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
-                         softmax_scale, sel_idx, scores, workspace, workspace_bytes, stream);
-  if (st) return st;
-  return sparse_decode_impl(shape, dtype, mode, q, K, V, mean_k, mean_v, count, sel_idx,
-                            budget_tokens, softmax_scale, out, workspace, workspace_bytes, stream,
-                            true);
+  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
+                           softmax_scale, sel_idx, scores, workspace, workspace_bytes, stream,
+                           Upto::kAttend, K, V, out);
 }
 
 int compkv_full_decode(const compkv_shape* shape, compkv_dtype dtype, const void* q,

@@ -260,6 +260,7 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* sh, int& total) {
 struct RadixCut {
   uint32_t prefix, mask;
   int quota;
+  bool whole;  // every key of the bucket is kept (no tie ranking needed)
 };
 
 template <typename KeyAt>
@@ -324,6 +325,148 @@ __device__ RadixCut cta_radix_cut(KeyAt key_at, int n, int K, uint32_t* hist, ui
   return RadixCut{prefix, mask, static_cast<int>(k)};
 }
 
+// Same contract as cta_radix_cut, tuned for non-negative float score keys: the first digit is
+// the top 11 bits (sign, exponent and two mantissa bits), which spreads scores over hundreds of
+// buckets, so the bucket holding the K-th largest key usually is selected whole after one pass.
+// Later digits take 8, 8 and 5 bits. Each pass: one barrier after counting, one inside the
+// block-wide scan of the bucket counts (in descending bucket order), one to publish the bucket.
+// `hist` holds 2592 uints (2048 + 256 + 256 + 32 buckets), `bc` 4 uints.
+namespace detail {
+// One digit pass of cta_topk_cut over NB = 2^BITS buckets at bit SHIFT (see there).
+template <int SHIFT, int BITS, typename KeyAt>
+__device__ __forceinline__ bool topk_pass(KeyAt key_at, int n, uint32_t* H, uint32_t* bc, int* sh,
+                                          uint32_t& prefix, uint32_t& mask, uint32_t& k) {
+  constexpr int NB = 1 << BITS;
+  constexpr uint32_t DM = NB - 1;
+  constexpr int PER = (NB + kThreads - 1) / kThreads;  // buckets per thread: 8 or 1
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const uint32_t key = key_at(i);
+    if ((key & mask) == prefix) atomicAdd(&H[(key >> SHIFT) & DM], 1u);
+  }
+  __syncthreads();
+  // descending scan: thread t owns buckets NB-1-t*PER ... NB-(t+1)*PER (first = highest)
+  uint32_t c[PER];
+  const int top = NB - 1 - static_cast<int>(threadIdx.x) * PER;
+  if constexpr (PER == 8) {
+    const uint4 lo = reinterpret_cast<const uint4*>(H + top - 7)[0];
+    const uint4 hi = reinterpret_cast<const uint4*>(H + top - 7)[1];
+    c[0] = hi.w; c[1] = hi.z; c[2] = hi.y; c[3] = hi.x; c[4] = lo.w; c[5] = lo.z; c[6] = lo.y; c[7] = lo.x;
+  } else {
+    c[0] = top >= 0 ? H[top] : 0u;
+  }
+  uint32_t cnt = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) cnt += c[e];
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sh[warp] = static_cast<int>(incl);
+  __syncthreads();
+  uint32_t base = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) base += (w < warp) ? static_cast<uint32_t>(sh[w]) : 0u;
+  const uint32_t excl = base + incl - cnt;
+  if (cnt > 0 && excl < k && k <= excl + cnt) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      if (run < k && run + c[e] >= k) {
+        bc[0] = static_cast<uint32_t>(top - e);
+        bc[1] = k - run;
+        bc[2] = c[e];
+      }
+      run += c[e];
+    }
+  }
+  __syncthreads();
+  const uint32_t bin = bc[0], bcnt = bc[2];
+  k = bc[1];
+  prefix |= bin << SHIFT;
+  mask |= DM << SHIFT;
+  return bcnt == k;  // the whole bucket is in the top K
+}
+}  // namespace detail
+
+// Same contract as cta_radix_cut, tuned for non-negative float score keys: the first digit is
+// the top 11 bits (sign, exponent and two mantissa bits), which spreads scores over hundreds of
+// buckets, so the bucket holding the K-th largest key usually is selected whole after one or two
+// passes. Later digits take 8, 8 and 5 bits. `hist` holds 2592 uints (2048 + 256 + 256 + 32
+// buckets, 16-byte aligned), `bc` 4 uints, `sh` kWarps ints. Two CTA barriers per pass.
+template <typename KeyAt>
+__device__ RadixCut cta_topk_cut(KeyAt key_at, int n, int K, uint32_t* hist, uint32_t* bc, int* sh) {
+  for (int i = threadIdx.x; i < 2592 / 4; i += kThreads) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  uint32_t prefix = 0, mask = 0, k = static_cast<uint32_t>(K);
+  if (detail::topk_pass<21, 11>(key_at, n, hist, bc, sh, prefix, mask, k))
+    return RadixCut{prefix, mask, static_cast<int>(k), true};
+  if (detail::topk_pass<13, 8>(key_at, n, hist + 2048, bc, sh, prefix, mask, k))
+    return RadixCut{prefix, mask, static_cast<int>(k), true};
+  if (detail::topk_pass<5, 8>(key_at, n, hist + 2304, bc, sh, prefix, mask, k))
+    return RadixCut{prefix, mask, static_cast<int>(k), true};
+  const bool whole = detail::topk_pass<0, 5>(key_at, n, hist + 2560, bc, sh, prefix, mask, k);
+  return RadixCut{prefix, mask, static_cast<int>(k), whole};
+}
+
+// Warp-wise version of cta_select_ordered: warp w scans a contiguous run of items with its lanes
+// on consecutive items (no shared-memory bank conflicts), ballots give positions inside the warp
+// and one CTA barrier gives each warp's offset. `sh` needs 2 * kWarps ints.
+template <typename KeyAt, typename Emit>
+__device__ int cta_select_ordered_w(KeyAt key_at, int n, const RadixCut& cut, int* sh, Emit emit) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int span = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int i0 = warp * span, i1 = min(n, i0 + span);
+  const uint32_t lt = (1u << lane) - 1u;
+  int gt_w = 0, eq_w = 0;
+  for (int b = i0; b < i1; b += 32) {
+    const int i = b + lane;
+    const uint32_t km = i < i1 ? (key_at(i) & cut.mask) : 0u;
+    const bool valid = i < i1;
+    gt_w += __popc(__ballot_sync(0xffffffffu, valid && km > cut.prefix));
+    eq_w += __popc(__ballot_sync(0xffffffffu, valid && km == cut.prefix));
+  }
+  if (lane == 0) {
+    sh[warp] = gt_w;
+    sh[kWarps + warp] = eq_w;
+  }
+  __syncthreads();
+  int eq_before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const int e = sh[kWarps + w];
+    const int kept_w = sh[w] + (cut.whole ? e : max(0, min(e, cut.quota - eq_before)));
+    if (w < warp) total += kept_w;
+    eq_before += (w < warp) ? e : 0;
+  }
+  // total is now this warp's output offset
+  int pos = total, er = eq_before;
+  for (int b = i0; b < i1; b += 32) {
+    const int i = b + lane;
+    const bool valid = i < i1;
+    const uint32_t km = valid ? (key_at(i) & cut.mask) : 0u;
+    const bool gt = valid && km > cut.prefix, eq = valid && km == cut.prefix;
+    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+    const int my_er = er + __popc(beq & lt);
+    const bool keep = gt || (eq && (cut.whole || my_er < cut.quota));
+    const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+    if (keep) emit(i, pos + __popc(bk & lt));
+    pos += __popc(bk);
+    er += __popc(beq);
+  }
+  int kept_total = 0, eqb = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const int e = sh[kWarps + w];
+    kept_total += sh[w] + (cut.whole ? e : max(0, min(e, cut.quota - eqb)));
+    eqb += e;
+  }
+  __syncthreads();
+  return kept_total;
+}
+
 // Keeps item i if (key & mask) > prefix, or it equals prefix and fewer than `quota` such items
 // precede it; visits kept items in index order with their output position: emit(i, pos).
 // `sh` needs kWarps + 1 ints. Contains CTA barriers. Returns the number kept.
@@ -331,6 +474,15 @@ template <typename KeyAt, typename Emit>
 __device__ int cta_select_ordered(KeyAt key_at, int n, const RadixCut& cut, int* sh, Emit emit) {
   const int per = (n + kThreads - 1) / kThreads;
   const int i0 = min(n, static_cast<int>(threadIdx.x) * per), i1 = min(n, i0 + per);
+  if (cut.whole) {  // no ties to rank: keep every key at or above the bucket, one scan
+    int kept = 0;
+    for (int i = i0; i < i1; ++i) kept += ((key_at(i) & cut.mask) >= cut.prefix);
+    int kept_total;
+    int pos = cta_exclusive_scan(kept, sh, kept_total);
+    for (int i = i0; i < i1; ++i)
+      if ((key_at(i) & cut.mask) >= cut.prefix) emit(i, pos++);
+    return kept_total;
+  }
   int eq = 0, gt = 0;
   for (int i = i0; i < i1; ++i) {
     const uint32_t km = key_at(i) & cut.mask;

@@ -1,0 +1,731 @@
+// a1 (second half) + a2 + a3. Normalised group score, Top-K selection, and exact attention over
+// the selected blocks with Mean compensation of every omitted block, in one softmax (CompKV
+// abstract: exact attention over a selected subset, compensation of the omitted tail; review,
+// Summary: blocks selected up to a token budget by the compensation-aware score, "omitted blocks
+// contribute their block-mean logit").
+//
+// Runs after the streaming kernel, whose outputs it reads from the workspace: per-block log
+// scores u_{j,h}, per-block records {x_h = s q_h . mu_j + log n_j, n_j}, and per-segment partials
+// of log Zhat and of the compensation sum over all blocks.
+//
+// One thread-block cluster of C CTAs per (sequence, kv-head); rank c owns the blocks
+// [c*chunk, c*chunk + chunk):
+//  1. log Zhat_h (log-sum-exp over the segments), S_j = sum_h exp(u_{j,h} - log Zhat_h) for the
+//     rank's blocks as order-preserving uint32 keys (empty blocks key 0), and the rank's local
+//     Top-K_b under (S desc, index asc) by radix cut.
+//  2. Rank 0 gathers the C candidate lists over distributed shared memory (ascending block order)
+//     and cuts the global Top-K_b from them; the global Top-K_b under this strict order always
+//     lies inside the union of the local ones, so the result is exact. Meanwhile the other ranks
+//     merge the compensation partials of the kv-head's segments, a slice of channels each.
+//  3. Rank c attends the c-th contiguous slice of rank 0's ordered selection (balanced whatever
+//     the blocks' positions): bulk copies of their K and V rows (up to the
+//     cache capacity; rows past the block's token count are masked) and of their mean values,
+//     exact logits, an online softmax per head, P.V, and removal of the blocks' compensation terms
+//     (taken against the running max of the exact logits, which is at least every processed
+//     block's mean logit, so nothing overflows; a block's compensation mass never exceeds its
+//     exact mass, so the removal cancels at most what it adds).
+//  4. Rank 0 merges the ranks' partials with the compensation partial.
+// Flags run steps 1-2 only (score/select call) or steps 3-4 only on a given selection (sparse
+// decode call). Launched with programmatic dependent launch: the prologue overlaps the previous
+// kernel's tail.
+#include <cooperative_groups.h>
+
+#include <mutex>
+
+#include "attend.cuh"
+#include "common.cuh"
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace compkv {
+namespace {
+
+constexpr int kMaxCluster = 16;
+constexpr int kRound = 8;  // selected blocks per shared-memory round
+constexpr int kRows = kRound * kBlockTokens;
+
+__host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
+
+// Shared-memory layout, identical on host and device.
+struct FLay {
+  int chunk, ccap, gcap, slots;
+  size_t keys, ck, ci, gk, gi, hist, bc, sh, misc, zm, zs, fm, fl, cslice, selm;
+  size_t q, kbuf, vbuf, nu, lg, pT, red, acc, cp, ml, blk, xr, pw, sc, fac, mbar, total;
+  __host__ __device__ void build(int chunk_, int Kb, int C, int slots_, int G, int D, int esz, int ksub) {
+    chunk = chunk_;
+    slots = slots_;
+    ccap = Kb < chunk ? Kb : chunk;
+    gcap = ccap * C;
+    size_t o = 0;
+    hist = o;   o = a16(o + sizeof(uint32_t) * 2592);
+    keys = o;   o = a16(o + sizeof(uint32_t) * chunk);
+    ck = o;     o = a16(o + sizeof(uint32_t) * (ccap + 1));
+    ci = o;     o = a16(o + sizeof(int) * (ccap + 1));
+    gk = o;     o = a16(o + sizeof(uint32_t) * (gcap + 1));
+    gi = o;     o = a16(o + sizeof(int) * (gcap + 1));
+    bc = o;     o = a16(o + sizeof(uint32_t) * 4);
+    sh = o;     o = a16(o + sizeof(int) * 2 * kWarps);
+    misc = o;   o = a16(o + sizeof(int) * 96);
+    zm = o;     o = a16(o + sizeof(float) * slots * G);
+    zs = o;     o = a16(o + sizeof(float) * slots * G);
+    fm = o;     o = a16(o + sizeof(float) * slots * G);
+    fl = o;     o = a16(o + sizeof(float) * slots * G);
+    cslice = o; o = a16(o + sizeof(float) * G * D);
+    selm = o;   o = a16(o + sizeof(int) * (Kb + 1));
+    q = o;      o = a16(o + sizeof(float) * G * D);
+    kbuf = o;   o = a16(o + static_cast<size_t>(esz) * kRows * D);
+    vbuf = o;   o = a16(o + static_cast<size_t>(esz) * kRows * D);
+    nu = o;     o = a16(o + sizeof(float) * kRound * D);
+    lg = o;     o = a16(o + sizeof(float) * G * kRows);
+    pT = o;     o = a16(o + sizeof(float) * G * kRows);
+    red = o;    o = a16(o + sizeof(float) * (ksub * G * D > 256 ? ksub * G * D : 256));
+    acc = o;    o = a16(o + sizeof(float) * G * D);
+    cp = o;     o = a16(o + sizeof(float) * G * (D + 2));
+    ml = o;     o = a16(o + sizeof(float) * 16);
+    blk = o;    o = a16(o + sizeof(int) * 2 * kRound);
+    xr = o;     o = a16(o + sizeof(float) * G * kRound);
+    pw = o;     o = a16(o + sizeof(float) * G * kRound);
+    sc = o;     o = a16(o + sizeof(float) * 8);
+    fac = o;    o = a16(o + sizeof(float) * G * 34);
+    mbar = o;   o = a16(o + 8 * 2);
+    total = o;
+  }
+};
+
+struct FParams {
+  FLay L;
+  int mode, do_select, do_attend;
+  int Nb, Kb, T, chunk, bpc, slots, nctas_stream, tiles_per_pair, total_tiles;
+  float scale;
+  const void* q;
+  const void* K;
+  const void* V;
+  const float* mean_v;
+  const float* u;
+  const float* xrec;
+  const float* zpart;
+  const float* comp_seg;
+  float* comp;        // merged compensation partial [pairs][G][D+2] (written by select-only,
+                      // read by attend-only)
+  int32_t* sel_idx;   // [pairs][Kb]: written by select, read by attend-only
+  float* scores;
+  float* out;
+  int32_t* status;
+};
+
+__device__ __forceinline__ int stream_cta_of_tile(long long f, int nctas, int F) {
+  return static_cast<int>(((f + 1) * nctas - 1) / F);
+}
+
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_constant__ FParams p) {
+  using RG = RowGeom<T, D>;
+  using PVt = PV<T, D, G>;
+  constexpr int EPV = RG::kEpv, VEC = PVt::kVec;
+  constexpr int XS = xrec_stride(G);
+  extern __shared__ __align__(128) unsigned char sm[];
+  const FLay& L = p.L;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int pr = blockIdx.x / C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool compensate = p.mode != COMPKV_MODE_MASS;
+
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sm + L.hist);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + L.keys);
+  uint32_t* ck = reinterpret_cast<uint32_t*>(sm + L.ck);
+  int* ci = reinterpret_cast<int*>(sm + L.ci);
+  uint32_t* gk = reinterpret_cast<uint32_t*>(sm + L.gk);
+  int* gi = reinterpret_cast<int*>(sm + L.gi);
+  uint32_t* bc = reinterpret_cast<uint32_t*>(sm + L.bc);
+  int* shs = reinterpret_cast<int*>(sm + L.sh);
+  int* misc = reinterpret_cast<int*>(sm + L.misc);  // [0] candidates [1] gathered [6] selected [24..] gather offsets
+  float* logz = reinterpret_cast<float*>(misc + 64);  // [8]
+  float* cM = logz + 8;                               // [8] compensation max per head
+  float* cl = logz + 16;                              // [8] compensation sum per head
+  float* zm_s = reinterpret_cast<float*>(sm + L.zm);
+  float* zs_s = reinterpret_cast<float*>(sm + L.zs);
+  float* fm_s = reinterpret_cast<float*>(sm + L.fm);
+  float* fl_s = reinterpret_cast<float*>(sm + L.fl);
+  float* cslice = reinterpret_cast<float*>(sm + L.cslice);
+  int* selm = reinterpret_cast<int*>(sm + L.selm);
+  float* q_s = reinterpret_cast<float*>(sm + L.q);
+  T* kbuf = reinterpret_cast<T*>(sm + L.kbuf);
+  T* vbuf = reinterpret_cast<T*>(sm + L.vbuf);
+  float* nu_s = reinterpret_cast<float*>(sm + L.nu);
+  float* lg = reinterpret_cast<float*>(sm + L.lg);
+  float* pT = reinterpret_cast<float*>(sm + L.pT);
+  float* red = reinterpret_cast<float*>(sm + L.red);
+  float* acc_s = reinterpret_cast<float*>(sm + L.acc);
+  float* cp_s = reinterpret_cast<float*>(sm + L.cp);
+  float* ml_s = reinterpret_cast<float*>(sm + L.ml);
+  int* blk_j = reinterpret_cast<int*>(sm + L.blk);
+  int* blk_n = blk_j + kRound;
+  float* xr_s = reinterpret_cast<float*>(sm + L.xr);
+  float* pw_s = reinterpret_cast<float*>(sm + L.pw);
+  float* sc_s = reinterpret_cast<float*>(sm + L.sc);
+  float* fac_s = reinterpret_cast<float*>(sm + L.fac);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L.mbar);
+
+  // ---- prologue (inputs written before the streaming kernel started)
+  if (tid == 0) {
+    mbar_init(&mbar[0], 1);
+    mbar_init_fence();
+  }
+  if (p.do_attend) {
+    const T* qp = static_cast<const T*>(p.q) + static_cast<size_t>(pr) * G * D;
+    for (int i = tid; i < G * D; i += kThreads) q_s[i] = to_float(qp[i]);
+  }
+  __syncthreads();
+  const int li = lane % RG::kLpr;
+  float qr[G][EPV];
+  if (p.do_attend) load_q_regs<T, D, G>(q_s, li, qr);
+
+  pdl_wait();  // the previous kernel's outputs are visible from here on
+
+  const int Kb = p.Kb;
+  const int j0 = rank * p.chunk;
+  const int nloc = max(0, min(p.chunk, p.Nb - j0));
+  int nsel = 0;
+
+  if (p.do_select) {
+    const long long f_first = static_cast<long long>(pr) * p.tiles_per_pair;
+    const int c_first = stream_cta_of_tile(f_first, p.nctas_stream, p.total_tiles);
+    const int nseg = stream_cta_of_tile(f_first + p.tiles_per_pair - 1, p.nctas_stream, p.total_tiles) - c_first + 1;
+    const float* zp = p.zpart + static_cast<size_t>(pr) * p.slots * G * 2;
+    const float* cs = p.comp_seg + static_cast<size_t>(pr) * p.slots * G * (D + 2);
+    const float* up = p.u + (static_cast<size_t>(pr) * p.Nb + j0) * G;
+    // ---- 1a. segment partials (one round trip); per-block log scores stay in flight meanwhile
+    for (int t = tid; t < nseg * G; t += kThreads) {
+      zm_s[t] = zp[2 * t];
+      zs_s[t] = zp[2 * t + 1];
+      if (compensate) {
+        fm_s[t] = cs[static_cast<size_t>(t) * (D + 2)];
+        fl_s[t] = cs[static_cast<size_t>(t) * (D + 2) + 1];
+      }
+    }
+    constexpr int UPT = 4;  // log-score rows prefetched per thread before log Zhat is known
+    float ur[UPT][G];
+#pragma unroll
+    for (int k = 0; k < UPT; ++k) {
+      const int j = tid + k * kThreads;
+#pragma unroll
+      for (int h = 0; h < G; ++h) ur[k][h] = (j < nloc) ? up[static_cast<size_t>(j) * G + h] : 0.f;
+    }
+    __syncthreads();
+    // ---- 1b. log Zhat per head; compensation max, factors and sum per head
+    if (warp < G) {
+      const int h = warp;
+      float m = -CUDART_INF_F, s = 0.f;
+      for (int t = lane; t < nseg; t += 32) lse_merge(m, s, zm_s[t * G + h], zs_s[t * G + h]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        lse_merge(m, s, m2, s2);
+      }
+      if (lane == 0) logz[h] = (m == -CUDART_INF_F) ? -CUDART_INF_F : m + logf(s);
+      if (compensate) {
+        float M = -CUDART_INF_F;
+        for (int t = lane; t < nseg; t += 32) M = fmaxf(M, fm_s[t * G + h]);
+        M = warp_max(M);
+        float l = 0.f;
+        for (int t = lane; t < nseg; t += 32) {
+          const float mt = fm_s[t * G + h];
+          const float f = (mt == -CUDART_INF_F) ? 0.f : __expf(mt - M);
+          fm_s[t * G + h] = f;
+          l = fmaf(f, fl_s[t * G + h], l);
+        }
+        l = warp_sum(l);
+        if (lane == 0) {
+          cM[h] = M;
+          cl[h] = l;
+        }
+      }
+    }
+    __syncthreads();
+    // ---- 1c. keys of this rank's blocks
+    float lz[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) lz[h] = logz[h];
+    for (int k = 0, j = tid; j < nloc; ++k, j += kThreads) {
+      float S = 0.f;
+      if (k < UPT) {
+#pragma unroll
+        for (int kk = 0; kk < UPT; ++kk)
+          if (kk == k) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) S += __expf(ur[kk][h] - lz[h]);
+          }
+      } else {
+#pragma unroll
+        for (int h = 0; h < G; ++h) S += __expf(up[static_cast<size_t>(j) * G + h] - lz[h]);
+      }
+      const bool empty = S != S;
+      keys[j] = empty ? 0u : score_key(S);
+      if (p.scores) p.scores[static_cast<size_t>(pr) * p.Nb + j0 + j] = empty ? 0.f : S;
+    }
+    __syncthreads();
+    // ---- 1d. local Top-K_b candidates, in ascending block order
+    if (tid == 0) misc[0] = 0;
+    if (Kb > 0) {
+      int ncand;
+      if (nloc <= Kb) {
+        for (int j = tid; j < nloc; j += kThreads) {
+          ck[j] = keys[j];
+          ci[j] = j0 + j;
+        }
+        ncand = nloc;
+      } else {
+        auto kat = [&](int i) { return keys[i]; };
+        const RadixCut cut = cta_topk_cut(kat, nloc, Kb, hist, bc, shs);
+        ncand = cta_select_ordered_w(kat, nloc, cut, shs, [&](int i, int pos) {
+          ck[pos] = keys[i];
+          ci[pos] = j0 + i;
+        });
+      }
+      if (tid == 0) misc[0] = ncand;
+    }
+    cluster.sync();  // #1: every rank's candidates are visible
+
+    // ---- 2. rank 0: global cut over the gathered candidates; other ranks: compensation merge
+    if (rank == 0 && Kb > 0) {
+      if (tid < C) misc[24 + tid] = *cluster.map_shared_rank(&misc[0], tid);
+      __syncthreads();
+      if (tid == 0) {
+        int off = 0;
+        for (int c = 0; c < C; ++c) {
+          const int n = misc[24 + c];
+          misc[24 + c] = off;
+          off += n;
+        }
+        misc[24 + C] = off;
+        misc[1] = off;
+      }
+      __syncthreads();
+      const int M = misc[1];
+      for (int i = tid; i < M; i += kThreads) {
+        int c = 0;
+        while (c + 1 < C && misc[24 + c + 1] <= i) ++c;
+        const int k = i - misc[24 + c];
+        gk[i] = *cluster.map_shared_rank(&ck[k], c);
+        gi[i] = *cluster.map_shared_rank(&ci[k], c);
+      }
+      __syncthreads();
+      auto kat = [&](int i) { return gk[i]; };
+      RadixCut cut{0u, 0u, M, true};  // fewer candidates than K_b: keep them all
+      if (M > Kb) cut = cta_topk_cut(kat, M, Kb, hist, bc, shs);
+      int32_t* sel = p.sel_idx ? p.sel_idx + static_cast<size_t>(pr) * Kb : nullptr;
+      const int nout = cta_select_ordered_w(kat, M, cut, shs, [&](int i, int pos) {
+        selm[pos] = gi[i];
+        if (sel) sel[pos] = gi[i];
+      });
+      if (tid == 0) misc[6] = nout;
+    }
+    if (compensate && (C == 1 || rank != 0)) {
+      // merge a slice of the compensation partials' channels: lanes along channels (coalesced),
+      // 4 segment groups summed in a fixed order
+      const int E = G * D, W = (C == 1) ? 1 : C - 1, wr = (C == 1) ? 0 : rank - 1;
+      const int per = (E + W - 1) / W;
+      const int e0 = wr * per, e1 = min(E, e0 + per);
+      float* mrg = red;  // scratch (the attention has not started)
+      const int ei = tid % 64, sg = tid / 64;
+      for (int base = e0; base < e1; base += 64) {
+        const int e = base + ei;
+        float a = 0.f;
+        if (e < e1) {
+          const int h = e / D, c = e % D;
+#pragma unroll 8
+          for (int t = sg; t < nseg; t += 4)
+            a = fmaf(fm_s[t * G + h], cs[(static_cast<size_t>(t) * G + h) * (D + 2) + 2 + c], a);
+        }
+        mrg[sg * 64 + ei] = a;
+        __syncthreads();
+        if (tid < 64 && base + tid < e1) {
+          const int e2 = base + tid;
+          const float v = ((mrg[tid] + mrg[64 + tid]) + mrg[128 + tid]) + mrg[192 + tid];
+          cslice[e2] = v;
+          if (!p.do_attend) p.comp[(static_cast<size_t>(pr) * G + e2 / D) * (D + 2) + 2 + (e2 % D)] = v;
+        }
+        __syncthreads();
+      }
+    }
+    if (compensate && !p.do_attend && rank == 0 && tid < G) {
+      float* o = p.comp + (static_cast<size_t>(pr) * G + tid) * (D + 2);
+      o[0] = cM[tid];
+      o[1] = cl[tid];
+    }
+    cluster.sync();  // #2: the cut and the merged compensation slices are visible
+
+    // ---- 3a. this rank's share of the selection: a contiguous slice of rank 0's ordered list
+    if (p.do_attend && Kb > 0) {
+      const int total = *cluster.map_shared_rank(&misc[6], 0);
+      const int per = (total + C - 1) / C;
+      const int s0 = min(total, rank * per), s1 = min(total, s0 + per);
+      if (rank != 0) {
+        const int* sel0 = cluster.map_shared_rank(selm, 0);
+        for (int i = tid; i < s1 - s0; i += kThreads) selm[i] = sel0[s0 + i];
+      }
+      nsel = s1 - s0;
+      __syncthreads();
+    }
+  }
+  if (!p.do_select && p.do_attend) {  // attend a given selection: rank c takes a slice of slots
+    const int s0 = min(Kb, rank * p.bpc), s1 = min(Kb, s0 + p.bpc);
+    for (int i = tid; i < s1 - s0; i += kThreads) selm[i] = p.sel_idx[static_cast<size_t>(pr) * Kb + s0 + i];
+    nsel = s1 - s0;
+    __syncthreads();
+  }
+  if (!p.do_attend) return;  // select only: no shared memory of another rank is read after #2
+
+  // compensation partial for the final merge (rank 0), fetched while the attention runs
+  if (rank == 0 && compensate) {
+    if (p.do_select) {
+      const int E = G * D, W = (C == 1) ? 1 : C - 1, per = (E + W - 1) / W;
+      for (int e = tid; e < E; e += kThreads) {
+        const int owner = (C == 1) ? 0 : 1 + e / per;
+        cp_s[(e / D) * (D + 2) + 2 + (e % D)] = *cluster.map_shared_rank(&cslice[e], owner);
+      }
+      if (tid < G) {
+        cp_s[tid * (D + 2)] = cM[tid];
+        cp_s[tid * (D + 2) + 1] = cl[tid];
+      }
+    } else {
+      const float* cp = p.comp + static_cast<size_t>(pr) * G * (D + 2);
+      for (int i = tid; i < G * (D + 2); i += kThreads) cp_s[i] = cp[i];
+    }
+  }
+
+  // ---- 3b. exact attention over this rank's selected blocks, in rounds of kRound blocks
+  const T* Kbase = static_cast<const T*>(p.K) + static_cast<size_t>(pr) * p.T * D;
+  const T* Vbase = static_cast<const T*>(p.V) + static_cast<size_t>(pr) * p.T * D;
+  const float* NUbase = p.mean_v + static_cast<size_t>(pr) * p.Nb * D;
+  const float* XRbase = p.xrec + static_cast<size_t>(pr) * p.Nb * XS;
+  const int cv = tid % PVt::kCols, sub = tid / PVt::kCols;
+  float acc[G][VEC];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
+  float m_run = -CUDART_INF_F, l_run = 0.f;  // warp h's running state for head h
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (int rs0 = 0; rs0 < nsel; rs0 += kRound) {
+    const int nr = min(kRound, nsel - rs0);
+    if (tid < kRound) {
+      int j = (tid < nr) ? selm[rs0 + tid] : -1;
+      if (j < 0 || j >= p.Nb) j = -1;
+      blk_j[tid] = j;
+    }
+    __syncthreads();
+    if (tid == 0) {  // K and V rows up to the cache capacity; the token count comes with the record
+      uint32_t bytes = 0;
+      for (int s2 = 0; s2 < nr; ++s2) {
+        const int j = blk_j[s2];
+        if (j < 0) continue;
+        const int rows = min(kBlockTokens, p.T - j * kBlockTokens);
+        bytes += 2u * rows * D * sizeof(T) + (compensate ? D * sizeof(float) : 0u);
+      }
+      mbar_arrive_expect_tx(&mbar[0], bytes);
+      for (int s2 = 0; s2 < nr; ++s2) {
+        const int j = blk_j[s2];
+        if (j < 0) continue;
+        const int rows = min(kBlockTokens, p.T - j * kBlockTokens);
+        const size_t off = static_cast<size_t>(j) * kBlockTokens * D;
+        bulk_g2s(kbuf + s2 * kBlockTokens * D, Kbase + off, rows * D * sizeof(T), &mbar[0]);
+        bulk_g2s(vbuf + s2 * kBlockTokens * D, Vbase + off, rows * D * sizeof(T), &mbar[0]);
+        if (compensate) bulk_g2s(nu_s + s2 * D, NUbase + static_cast<size_t>(j) * D, D * sizeof(float), &mbar[0]);
+      }
+    }
+    if (tid < nr * (G + 1)) {  // records: x_h and the token count of each block
+      const int s2 = tid / (G + 1), e = tid % (G + 1);
+      const int j = blk_j[s2];
+      const float v = (j >= 0) ? XRbase[static_cast<size_t>(j) * XS + e] : 0.f;
+      if (e < G) xr_s[s2 * G + e] = (j >= 0) ? v : -CUDART_INF_F;
+      else blk_n[s2] = (j >= 0) ? max(0, min(__float_as_int(v), min(kBlockTokens, p.T - j * kBlockTokens))) : 0;
+    }
+    if (tid >= nr && tid < kRound) blk_n[tid] = 0;
+    const bool got = mbar_wait(&mbar[0], phase, p.status);
+    __syncthreads();  // records visible
+    for (int s2 = 0; s2 < nr; ++s2) {  // V rows past a block's token count: zero (0 * NaN is NaN)
+      const int n = blk_n[s2];
+      if (n < kBlockTokens) {
+        T* vrow = vbuf + (static_cast<size_t>(s2) * kBlockTokens + n) * D;
+        for (int e = tid; e < (kBlockTokens - n) * D; e += kThreads) vrow[e] = T(0);
+      }
+    }
+    fence_proxy_async();  // the next round's copies may land on these rows
+    if (__syncthreads_and(got) == 0) {  // uniform: drain (bounded) and stop
+      mbar_wait(&mbar[0], phase, nullptr);
+      break;
+    }
+    phase ^= 1;
+    const int R = nr * kBlockTokens;
+    const int Rpad = (R + kWarps * RG::kRpl - 1) / (kWarps * RG::kRpl) * (kWarps * RG::kRpl);
+    tile_logits<T, D, G>(kbuf, Rpad, qr, p.scale, lg, kRows, [&](int row) {
+      return row < R && (row % kBlockTokens) < blk_n[row / kBlockTokens];
+    });
+    __syncthreads();
+    if (warp < G) {  // softmax update for head h; compensation terms of these blocks removed
+      const int h = warp;
+      float mx = -CUDART_INF_F;
+      for (int row = lane; row < R; row += 32) mx = fmaxf(mx, lg[h * kRows + row]);
+      mx = warp_max(mx);
+      const float m_new = fmaxf(m_run, mx);
+      float ls = 0.f;
+      for (int row = lane; row < R; row += 32) {
+        const float x = lg[h * kRows + row];
+        const float w = (x == -CUDART_INF_F) ? 0.f : __expf(x - m_new);
+        pT[row * G + h] = w;
+        ls += w;
+      }
+      ls = warp_sum(ls);
+      float pw = 0.f;
+      if (compensate && lane < nr) {
+        const float xj = xr_s[lane * G + h];
+        pw = (xj == -CUDART_INF_F) ? 0.f : __expf(xj - m_new);
+      }
+      if (lane < kRound) pw_s[h * kRound + lane] = pw;
+      const float pws = warp_sum(pw);
+      const float scl = (m_run == -CUDART_INF_F) ? 0.f : __expf(m_run - m_new);
+      l_run = l_run * scl + ls - pws;
+      m_run = m_new;
+      if (lane == 0) sc_s[h] = scl;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float scl = sc_s[h];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[h][e] *= scl;
+    }
+    PVt::accumulate(vbuf, pT, R, sub, cv, acc);
+    if (compensate && sub == 0) {
+      for (int s2 = 0; s2 < nr; ++s2) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float nv = nu_s[s2 * D + cv * VEC + e];
+#pragma unroll
+          for (int h = 0; h < G; ++h) acc[h][e] = fmaf(-pw_s[h * kRound + s2], nv, acc[h][e]);
+        }
+      }
+    }
+    __syncthreads();  // buffers are reused by the next round
+  }
+
+  // ---- this rank's partial (m, l, acc) per head -> shared memory
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[(sub * G + h) * D + cv * VEC + e] = acc[h][e];
+  if (warp < G && lane == 0) {
+    ml_s[2 * warp] = m_run;
+    ml_s[2 * warp + 1] = l_run;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kThreads) {
+    float sum = 0.f;
+    for (int k = 0; k < PVt::kSub; ++k) sum += red[k * G * D + i];
+    acc_s[i] = sum;
+  }
+  cluster.sync();  // #3: every rank's partial is visible
+
+  // ---- 4. rank 0 merges the ranks' partials and the compensation partial
+  if (rank == 0) {
+    if (tid < G * C) {
+      const int h = tid / C, s2 = tid % C;
+      const float* rml = cluster.map_shared_rank(ml_s, s2);
+      fac_s[h * 17 + s2] = rml[2 * h];
+      fac_s[G * 17 + h * 17 + s2] = rml[2 * h + 1];
+    }
+    __syncthreads();
+    if (tid < G) {
+      const int h = tid;
+      const float cmh = compensate ? cp_s[h * (D + 2)] : -CUDART_INF_F;
+      float M = cmh;
+      for (int s2 = 0; s2 < C; ++s2) M = fmaxf(M, fac_s[h * 17 + s2]);
+      float den = 0.f;
+      if (cmh != -CUDART_INF_F) {
+        const float f = __expf(cmh - M);
+        fac_s[h * 17 + 16] = f;
+        den = f * cp_s[h * (D + 2) + 1];
+      } else {
+        fac_s[h * 17 + 16] = 0.f;
+      }
+      for (int s2 = 0; s2 < C; ++s2) {
+        const float ms = fac_s[h * 17 + s2];
+        const float f = (ms == -CUDART_INF_F) ? 0.f : __expf(ms - M);
+        fac_s[h * 17 + s2] = f;
+        den = fmaf(f, fac_s[G * 17 + h * 17 + s2], den);
+      }
+      sc_s[h] = den > 0.f ? 1.f / den : 0.f;
+    }
+    __syncthreads();
+    float* o = p.out + static_cast<size_t>(pr) * G * D;
+    for (int i = tid; i < G * D; i += kThreads) {
+      const int h = i / D, c = i % D;
+      float part[kMaxCluster];
+#pragma unroll
+      for (int s2 = 0; s2 < kMaxCluster; ++s2) part[s2] = (s2 < C) ? cluster.map_shared_rank(acc_s, s2)[i] : 0.f;
+      float a = compensate ? fac_s[h * 17 + 16] * cp_s[h * (D + 2) + 2 + c] : 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < kMaxCluster; ++s2)
+        if (s2 < C) a = fmaf(fac_s[h * 17 + s2], part[s2], a);  // factors past C are not set
+      o[i] = a * sc_s[h];
+    }
+  }
+  cluster.sync();  // #4: rank 0 is done reading the other ranks' shared memory
+}
+
+template <typename T, int D>
+const void* kptr_g(int G) {
+  switch (G) {
+    case 1: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 1>);
+    case 2: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 2>);
+    case 4: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 4>);
+    case 8: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 8>);
+  }
+  return nullptr;
+}
+
+int ksub_of(bool bf16, int D) { return kThreads / (D / (bf16 ? 2 : 1)); }
+
+const void* pick(bool bf16, int D, int G) {
+  if (bf16) return D == 128 ? kptr_g<uint16_t, 128>(G) : (D == 64 ? kptr_g<uint16_t, 64>(G) : nullptr);
+  return D == 128 ? kptr_g<float, 128>(G) : (D == 64 ? kptr_g<float, 64>(G) : nullptr);
+}
+
+// Launch plan of one problem shape: the cluster size and the shared-memory layout.
+struct Plan {
+  const void* kern = nullptr;
+  int dev = -1, pairs = 0, Nb = 0, Kb = 0, slots = 0;
+  int C = 0, chunk = 0;
+  FLay L;
+};
+Plan g_plans[32];
+int g_nplans = 0, g_next = 0;
+std::mutex g_mu;
+
+cudaLaunchConfig_t make_cfg(int pairs, int C, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pairs * C, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cfg;
+}
+
+// Cluster size: the largest power of two <= 16 that keeps the grid within two CTAs per SM and
+// at least 64 blocks per rank, then the largest one the device can co-schedule.
+cudaError_t make_plan(const void* kern, const FusedArgs& a, Plan* out) {
+  int dev = 0, sms = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  int C0 = 1;
+  while (C0 < kMaxCluster && a.pairs * (2 * C0) <= 2 * sms && (a.Nb + 2 * C0 - 1) / (2 * C0) >= 64) C0 *= 2;
+  const int esz = a.bf16 ? 2 : 4;
+  for (int C = C0; C >= 1; C /= 2) {
+    const int chunk = (a.Nb + C - 1) / C;
+    FLay L;
+    L.build(chunk, a.Kb, C, a.slots, a.G, a.D, esz, ksub_of(a.bf16, a.D));
+    if (L.total > static_cast<size_t>(optin)) continue;
+    // the opt-in maximum, so that plans of different sizes share the kernel's attribute
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = make_cfg(a.pairs, C, L.total, nullptr, attr, false);
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      ncl = 0;
+    }
+    if (ncl >= 1) {
+      out->C = C;
+      out->chunk = chunk;
+      out->L = L;
+      return cudaSuccess;
+    }
+  }
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_fused(const FusedArgs& a, cudaStream_t st) {
+  const void* kern = pick(a.bf16, a.D, a.G);
+  if (!kern) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  Plan plan;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int found = -1;
+    for (int i = 0; i < g_nplans; ++i) {
+      const Plan& q = g_plans[i];
+      if (q.kern == kern && q.dev == dev && q.pairs == a.pairs && q.Nb == a.Nb && q.Kb == a.Kb && q.slots == a.slots)
+        found = i;
+    }
+    if (found >= 0) {
+      plan = g_plans[found];
+    } else {
+      cudaError_t e = make_plan(kern, a, &plan);
+      if (e != cudaSuccess) return e;
+      plan.kern = kern;
+      plan.dev = dev;
+      plan.pairs = a.pairs;
+      plan.Nb = a.Nb;
+      plan.Kb = a.Kb;
+      plan.slots = a.slots;
+      const int slot = g_nplans < 32 ? g_nplans++ : (g_next++ % 32);
+      g_plans[slot] = plan;
+    }
+  }
+  FParams p;
+  p.L = plan.L;
+  p.mode = a.mode;
+  p.do_select = a.do_select ? 1 : 0;
+  p.do_attend = a.do_attend ? 1 : 0;
+  p.Nb = a.Nb;
+  p.Kb = a.Kb;
+  p.T = a.T;
+  p.chunk = plan.chunk;
+  p.bpc = (a.Kb + plan.C - 1) / plan.C;
+  p.slots = a.slots;
+  p.nctas_stream = a.nctas_stream;
+  p.tiles_per_pair = (a.Nb + kStreamTile - 1) / kStreamTile;
+  p.total_tiles = a.pairs * p.tiles_per_pair;
+  p.scale = a.scale;
+  p.q = a.q;
+  p.K = a.K;
+  p.V = a.V;
+  p.mean_v = a.mean_v;
+  p.u = a.u;
+  p.xrec = a.xrec;
+  p.zpart = a.zpart;
+  p.comp_seg = a.comp_seg;
+  p.comp = a.comp;
+  p.sel_idx = a.sel_idx;
+  p.scores = a.scores;
+  p.out = a.out;
+  p.status = a.status;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = make_cfg(a.pairs, plan.C, plan.L.total, st, attr, a.pdl);
+  void* args[] = {&p};
+  return cudaLaunchKernelExC(&cfg, kern, args);
+}
+
+}  // namespace compkv

@@ -51,34 +51,30 @@ struct StreamArgs {
   int* nctas_out;    // grid size used (host), may be null
 };
 
-struct SelectArgs {
-  int mode;
-  int pairs, G, D, Nb, Kb, slots, nctas_stream;
-  const float* u;
-  const float* zpart;
-  const float* comp_seg;
-  float* comp;       // [pairs][G][D+2] merged compensation partial
-  int32_t* sel_idx;  // [pairs][Kb]
-  float* scores;     // [pairs][Nb] or null
-};
-
-struct SparseArgs {
+// The select-and-attend kernel (decode_fused.cu). do_select: Top-K_b from the streaming
+// kernel's outputs (writes sel_idx; without do_attend also the merged compensation partial
+// `comp`). do_attend: attention over the selection (with do_select, the one just made; without,
+// sel_idx and `comp` as given).
+struct FusedArgs {
   bool bf16;
   int mode;
-  int B, Hkv, G, D, T, Nb, Kb;
+  bool do_select, do_attend;
+  int pairs, G, D, T, Nb, Kb, slots, nctas_stream;
   float scale;
   const void* q;
   const void* K;
   const void* V;
-  const float* mean_k;
   const float* mean_v;
-  const int32_t* count;
-  const int32_t* sel_idx;
-  const float* comp;  // [B*Hkv][G][D+2] merged compensation partial
-  const float* xrec;  // [B*Hkv][Nb][xrec_stride(G)] from the streaming kernel
-  float* out;
+  const float* u;
+  const float* xrec;      // [pairs][Nb][xrec_stride(G)] from the streaming kernel
+  const float* zpart;
+  const float* comp_seg;
+  float* comp;            // [pairs][G][D+2] merged compensation partial
+  int32_t* sel_idx;       // [pairs][Kb]
+  float* scores;          // [pairs][Nb] or null
+  float* out;             // [pairs][G][D]
   int32_t* status;
-  bool pdl;           // launched right after the select kernel: programmatic dependent launch
+  bool pdl;               // launched right after the streaming kernel: programmatic dependent launch
 };
 
 struct FullArgs {
@@ -129,16 +125,13 @@ struct StepWorkspace {
 
 // Grid size of the streaming score kernel for this shape on the current device.
 int stream_grid_ctas(bool bf16, int D, int G, int r, int total_tiles);
-// Blocks per CTA and the CTA count per kv-head (a cluster) of sparse_decode.
-void sparse_split(int B, int Hkv, int Kb, int* blocks_per_cta, int* nsplit);
 // Splits per kv-head of full_decode (<= max_full_splits(T)).
 int full_splits(int B, int Hkv, int T);
 inline int max_full_splits(int T) { return (T + 511) / 512; }
 
 cudaError_t launch_build_summaries(const SummariesArgs& a, cudaStream_t st);
 cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st);
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
-cudaError_t launch_sparse_decode(const SparseArgs& a, cudaStream_t st);
+cudaError_t launch_decode_fused(const FusedArgs& a, cudaStream_t st);
 cudaError_t launch_full_decode(const FullArgs& a, cudaStream_t st);
 
 }  // namespace compkv

@@ -88,7 +88,8 @@ __device__ __forceinline__ float pick_h(const float (&a)[G], int h) {
   return v;
 }
 
-template <typename TQ, int D, int G>
+// R = 4 specialises the default group count (grouped variances as one float4); R = 0 is any r.
+template <typename TQ, int D, int G, int R>
 __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_constant__ StreamParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   SLay L;
@@ -155,14 +156,20 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   constexpr int LPH = LPB / G;          // lanes per head after the transpose-reduce
   constexpr int LR = D / 4;             // lanes per mean-value row (4 channels per lane)
   constexpr int RS = 32 / LR;           // mean-value rows per warp step
-  constexpr int NSL = kWarps * BPP;     // head lanes per head in the CTA
+  constexpr int NSL = kWarps * BPP * PASSES;  // scalar lanes per head in the CTA
+  static_assert(PASSES <= LPH, "scalar lanes of a block must cover its passes");
   const int li = lane % LPB, bsub = lane / LPB;
-  const bool head_lane = (li % LPH) == 0;
+  // after the transpose-reduce, lane li of a block group holds head li / LPH; the pass-p value is
+  // moved p lanes up, so lane (h * LPH + p) does the scalar work of (pass p, head h)
+  const int my_pass = li % LPH;
+  const bool head_lane = my_pass < PASSES;
   const int my_h = li / LPH;
+  const int my_bl = my_pass * BPP + bsub;  // block of this scalar lane within the warp's 4
   const int c4 = lane % LR, rsub = lane / LR;
-  const int slot = warp * BPP + bsub;
+  const int slot = (warp * BPP + bsub) * PASSES + my_pass;
 
-  float qreg[G][8];
+  float2 qreg[G][4];
+  float qnr[4];
   float acc[G][4];
   float mref[G];
   float zmax = -CUDART_INF_F, zsum = 0.f, lsum = 0.f;
@@ -244,15 +251,20 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       }
       qn_s[i] = p.scale * p.scale * s;
     }
+    __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
+      qreg[h][0] = make_float2(q_s[h * D + li * 4 + 0], q_s[h * D + li * 4 + 1]);
+      qreg[h][1] = make_float2(q_s[h * D + li * 4 + 2], q_s[h * D + li * 4 + 3]);
+      qreg[h][2] = make_float2(q_s[h * D + D / 2 + li * 4 + 0], q_s[h * D + D / 2 + li * 4 + 1]);
+      qreg[h][3] = make_float2(q_s[h * D + D / 2 + li * 4 + 2], q_s[h * D + D / 2 + li * 4 + 3]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        qreg[h][e] = q_s[h * D + li * 4 + e];
-        qreg[h][4 + e] = q_s[h * D + D / 2 + li * 4 + e];
-        acc[h][e] = 0.f;
-      }
+      for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
       mref[h] = -CUDART_INF_F;
+    }
+    if constexpr (R == 4) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) qnr[g] = qn_s[my_h * 4 + g];
     }
     zmax = -CUDART_INF_F;
     zsum = lsum = 0.f;
@@ -309,38 +321,46 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       const float4 b = reinterpret_cast<const float4*>(mu_t + jt * D + D / 2)[li];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float s = qreg[h][0] * a.x;
-        s = fmaf(qreg[h][1], a.y, s);
-        s = fmaf(qreg[h][2], a.z, s);
-        s = fmaf(qreg[h][3], a.w, s);
-        s = fmaf(qreg[h][4], b.x, s);
-        s = fmaf(qreg[h][5], b.y, s);
-        s = fmaf(qreg[h][6], b.z, s);
-        s = fmaf(qreg[h][7], b.w, s);
-        v[pass][h] = s;
+        float2 s2 = __fmul2_rn(qreg[h][0], make_float2(a.x, a.y));
+        s2 = __ffma2_rn(qreg[h][1], make_float2(a.z, a.w), s2);
+        s2 = __ffma2_rn(qreg[h][2], make_float2(b.x, b.y), s2);
+        s2 = __ffma2_rn(qreg[h][3], make_float2(b.z, b.w), s2);
+        v[pass][h] = s2.x + s2.y;
       }
     }
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) TransposeReduce<G, LPB / 2>::run(v[pass], li);
-
-    // ---- (2) per (block, head) scalars on the head lanes
-    float xs[PASSES];
-    bool need = false;
-    const float mh0 = pick_h<G>(mref, my_h);
+    float dot = v[0][0];
 #pragma unroll
-    for (int pass = 0; pass < PASSES; ++pass) {
-      const int jt = warp * kBlocksPerWarp + pass * BPP + bsub;
-      xs[pass] = -CUDART_INF_F;
+    for (int pass = 1; pass < PASSES; ++pass) {
+      const float t = __shfl_up_sync(0xffffffffu, v[pass][0], pass);
+      if (my_pass == pass) dot = t;
+    }
+
+    // ---- (2) per (block, head) scalars, one (block, head) per scalar lane
+    float xs = -CUDART_INF_F;
+    bool need = false;
+    {
+      const int jt = warp * kBlocksPerWarp + my_bl;
       if (head_lane && jt < tn) {
         const int n = cnt_t[jt];
-        float vh = 0.f;
-        for (int g = 0; g < r; ++g) vh = fmaf(qn_s[my_h * r + g], var_t[jt * r + g], vh);
-        const float lbar = p.scale * v[pass][0];
+        float vh;
+        if constexpr (R == 4) {
+          const float4 vv = reinterpret_cast<const float4*>(var_t)[jt];
+          vh = qnr[0] * vv.x;
+          vh = fmaf(qnr[1], vv.y, vh);
+          vh = fmaf(qnr[2], vv.z, vh);
+          vh = fmaf(qnr[3], vv.w, vh);
+        } else {
+          vh = 0.f;
+          for (int g = 0; g < r; ++g) vh = fmaf(qn_s[my_h * r + g], var_t[jt * r + g], vh);
+        }
+        const float lbar = p.scale * dot;
         const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jt;
-        float uu, x = -CUDART_INF_F;
+        float uu;
         if (n > 0) {
-          x = lbar + logn_s[min(n, 16)];
-          const float lm = x + __logf(1.f + 0.5f * vh);
+          xs = lbar + logn_s[min(n, 16)];
+          const float lm = xs + __logf(1.f + 0.5f * vh);
           uu = (p.mode == COMPKV_MODE_COMPKV) ? lm + __logf(0.5f * vh) : lm;
           if (lm > zmax) {
             zsum = zsum * __expf(zmax - lm) + 1.f;
@@ -348,13 +368,12 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
           } else {
             zsum += __expf(lm - zmax);
           }
-          need = need || (x > mh0 + kRefSlack);
+          need = xs > pick_h<G>(mref, my_h) + kRefSlack;
         } else {
           uu = __int_as_float(0x7fffffff);  // NaN marks an empty block
         }
-        xs[pass] = x;
         p.u[row * G + my_h] = uu;
-        p.xrec[row * XS + my_h] = x;
+        p.xrec[row * XS + my_h] = xs;
         if (my_h == 0) p.xrec[row * XS + G] = __int_as_float(n);
       }
     }
@@ -363,10 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
         float sc_mine = 1.f;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          float m = -CUDART_INF_F;
-#pragma unroll
-          for (int pass = 0; pass < PASSES; ++pass) m = fmaxf(m, (head_lane && my_h == h) ? xs[pass] : -CUDART_INF_F);
-          const float tm = warp_max(m);
+          const float tm = warp_max((head_lane && my_h == h) ? xs : -CUDART_INF_F);
           const float nm = (tm > mref[h] + kRefSlack) ? tm : mref[h];
           const float sc = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - nm);
           acc[h][0] *= sc; acc[h][1] *= sc; acc[h][2] *= sc; acc[h][3] *= sc;
@@ -375,14 +391,10 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
         }
         lsum *= sc_mine;
       }
-      const float mh = pick_h<G>(mref, my_h);
-#pragma unroll
-      for (int pass = 0; pass < PASSES; ++pass) {
-        const float w = (xs[pass] == -CUDART_INF_F) ? 0.f : __expf(xs[pass] - mh);
-        if (head_lane) {
-          wsw[(pass * BPP + bsub) * G + my_h] = w;
-          lsum += w;
-        }
+      if (head_lane) {
+        const float w = (xs == -CUDART_INF_F) ? 0.f : __expf(xs - pick_h<G>(mref, my_h));
+        wsw[my_bl * G + my_h] = w;
+        lsum += w;
       }
       __syncwarp();
       // ---- (3) acc_h += w_{j,h} nu_j over this warp's blocks: 4 channels x G heads per lane
@@ -395,10 +407,13 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float w = wsw[bl * G + h];
-            acc[h][0] = fmaf(w, nv.x, acc[h][0]);
-            acc[h][1] = fmaf(w, nv.y, acc[h][1]);
-            acc[h][2] = fmaf(w, nv.z, acc[h][2]);
-            acc[h][3] = fmaf(w, nv.w, acc[h][3]);
+            const float2 w2 = make_float2(w, w);
+            const float2 lo = __ffma2_rn(w2, make_float2(nv.x, nv.y), make_float2(acc[h][0], acc[h][1]));
+            const float2 hi = __ffma2_rn(w2, make_float2(nv.z, nv.w), make_float2(acc[h][2], acc[h][3]));
+            acc[h][0] = lo.x;
+            acc[h][1] = lo.y;
+            acc[h][2] = hi.x;
+            acc[h][3] = hi.y;
           }
         }
       }
@@ -415,17 +430,18 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
 }
 
 template <typename TQ, int D, int G>
-const void* kptr() {
-  return reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G>);
+const void* kptr(int r) {
+  return r == 4 ? reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G, 4>)
+                : reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G, 0>);
 }
 
-const void* pick(bool bf16, int D, int G) {
+const void* pick(bool bf16, int D, int G, int r) {
 #define COMPKV_PICK(T, DD)                  \
   switch (G) {                              \
-    case 1: return kptr<T, DD, 1>();        \
-    case 2: return kptr<T, DD, 2>();        \
-    case 4: return kptr<T, DD, 4>();        \
-    case 8: return kptr<T, DD, 8>();        \
+    case 1: return kptr<T, DD, 1>(r);       \
+    case 2: return kptr<T, DD, 2>(r);       \
+    case 4: return kptr<T, DD, 4>(r);       \
+    case 8: return kptr<T, DD, 8>(r);       \
   }
   if (bf16) {
     if (D == 128) { COMPKV_PICK(uint16_t, 128) } else { COMPKV_PICK(uint16_t, 64) }
@@ -483,7 +499,7 @@ int stream_ctas(int total_tiles, int sms, int ctas_per_sm) {
 }  // namespace
 
 cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
-  const void* kern = pick(a.bf16, a.D, a.G);
+  const void* kern = pick(a.bf16, a.D, a.G, a.r);
   if (!kern) return cudaErrorInvalidValue;
   Grid g;
   cudaError_t e = grid_for(kern, a.D, a.G, a.r, &g);
@@ -519,7 +535,7 @@ cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
 }
 
 int stream_grid_ctas(bool bf16, int D, int G, int r, int total_tiles) {
-  const void* kern = pick(bf16, D, G);
+  const void* kern = pick(bf16, D, G, r);
   Grid g;
   if (!kern || grid_for(kern, D, G, r, &g) != cudaSuccess) return -1;
   return stream_ctas(total_tiles, g.sms, g.ctas_per_sm);

@@ -3,8 +3,8 @@
 Sizes: the tiny case and shrunken Llama-layer caches that still span many 32-block tiles, several
 cluster ranks and a ragged tail run on every (b, kv-head); the full-size workloads (32K and 128K
 context, the 3 x 3 length/budget grid, the 16 x 64K batch) run in the launch configuration the
-benchmark times (decode_step: score/select then sparse decode with programmatic dependent
-launch) and are checked on sampled (b, kv-head) pairs the oracle computes one by one.
+benchmark times (decode_step: the streaming score kernel, then the select-and-attend kernel with
+programmatic dependent launch) and are checked on sampled (b, kv-head) pairs the oracle computes one by one.
 """
 import numpy as np
 import pytest
