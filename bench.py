@@ -248,7 +248,7 @@ def config_of(wl) -> dict:
             "input_dtype": wl.dtype, "summary_dtype": "fp32",
             "l2": f"rotates {N_CACHES} independent caches; working set "
                   f"{N_CACHES} x step bytes > 126 MB L2",
-            "graph": "CUDA graphs, score/select then sparse decode with programmatic dependent launch"}
+            "graph": "CUDA graphs; streaming score kernel, then the select-and-attend kernel with programmatic dependent launch"}
 
 
 # ---------------------------------------------------------------------------------- ours
