@@ -103,6 +103,21 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return p;
 }
 
+// Hint: bring the bytes [begin, begin + bytes) of global memory into L2 (no shared memory, no
+// completion to wait for). The range is shrunk inward to 16-byte boundaries, so nothing outside
+// it is touched. No multicast.
+__device__ __forceinline__ void prefetch_l2_range(const void* begin, size_t bytes) {
+  uintptr_t a = reinterpret_cast<uintptr_t>(begin);
+  uintptr_t e = a + bytes;
+  a = (a + 15) & ~static_cast<uintptr_t>(15);
+  e &= ~static_cast<uintptr_t>(15);
+  while (a < e) {
+    const uint32_t n = static_cast<uint32_t>((e - a) < (1u << 20) ? (e - a) : (1u << 20));
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
+    a += n;
+  }
+}
+
 // 4-byte asynchronous copy (any 4-byte aligned address); tracked by cp_async_arrive.
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)

@@ -13,16 +13,18 @@
 // bytes whatever B and Hkv are. A CTA's range crosses at most a few (sequence, kv-head) pairs; it
 // writes one partial record per pair it touches ("segment").
 //
-// Pipeline: a 3-stage shared-memory ring with a "full" and an "empty" mbarrier per stage. Warp 0
-// refills a stage (bulk copies of the tile's mean keys and mean values, 4-byte cp.async of its
-// grouped variances and counts) once all 8 warps have released it. Each warp owns 4 blocks of
-// every tile and works through the ring on its own, with no CTA barrier in steady state: its
-// lanes dot the mean keys with the G heads (transpose-reduce), the lane left holding head h's dot
-// does that (block, head)'s scalar work, and the warp accumulates its blocks' weighted mean
-// values for all G heads (4 channels per lane). Compensation weights are taken against a
+// Pipeline: a 3-stage shared-memory ring with a "full" mbarrier per stage. Each warp releases a
+// stage by bumping a shared counter; the last of the 8 to release it refills it at once (bulk
+// copies of the tile's mean keys and mean values, 4-byte cp.async of its grouped variances and
+// counts), so no warp waits to produce. Each warp owns 4 blocks of every tile and works through
+// the ring on its own, with no CTA barrier in steady state. Lane l holds the same VW channels of
+// every row for all G heads, so each mean key and mean value is read from shared memory once:
+// partial dots of the 4 blocks with the G heads, one transpose-reduce over the warp that leaves
+// each lane with one (block, head) dot for the scalar work, then each lane accumulates its
+// channels of every head's weighted mean values. Compensation weights are taken against a
 // per-warp reference logit per head that only moves up when a logit would exceed it by 64 (e^64
 // keeps every sum finite in fp32). Warps meet only where a segment ends, to merge their partials
-// in a fixed order (deterministic results).
+// in a fixed order (deterministic results), using the ring stage just released as scratch.
 //
 // Besides the log scores u it writes, per block, the record {x_h (h < G), n_j} that lets the
 // attention kernel add and remove the block's compensation term without re-reading its summary.
@@ -58,7 +60,7 @@ struct StreamParams {
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 struct SLay {
-  size_t stage_bytes, off_mu, off_nu, off_var, off_cnt, stage0, full, empty, wsw, q, qn, comp, refw, red, logn, total;
+  size_t stage_bytes, off_mu, off_nu, off_var, off_cnt, stage0, full, rel, wsw, q, qn, refw, red, logn, total;
   __host__ __device__ void build(int D, int G, int r) {
     off_mu = 0;
     off_nu = a16(sizeof(float) * kTile * D);
@@ -67,26 +69,17 @@ struct SLay {
     stage_bytes = a16(off_cnt + sizeof(int) * kTile);
     size_t o = 0;
     full = o;   o = a16(o + 8 * kStages);
-    empty = o;  o = a16(o + 8 * kStages);
-    stage0 = o; o = a16(o + stage_bytes * kStages);
+    rel = o;    o = a16(o + sizeof(uint32_t) * (kStages + 2));  // release counters, abort, issued
     wsw = o;    o = a16(o + sizeof(float) * kWarps * kBlocksPerWarp * G);   // per-warp weights
+    stage0 = o; o = a16(o + stage_bytes * kStages);
     q = o;      o = a16(o + sizeof(float) * G * D);
     qn = o;     o = a16(o + sizeof(float) * G * r);
-    comp = o;   o = a16(o + sizeof(float) * G * D);
     refw = o;   o = a16(o + sizeof(float) * kWarps * G);
     red = o;    o = a16(o + sizeof(float) * 3 * G * 32);
     logn = o;   o = a16(o + sizeof(float) * 17);
     total = o;
   }
 };
-
-template <int G>
-__device__ __forceinline__ float pick_h(const float (&a)[G], int h) {
-  float v = a[0];
-#pragma unroll
-  for (int i = 1; i < G; ++i) v = (h == i) ? a[i] : v;
-  return v;
-}
 
 // R = 4 specialises the default group count (grouped variances as one float4); R = 0 is any r.
 template <typename TQ, int D, int G, int R>
@@ -104,17 +97,17 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   constexpr int XS = xrec_stride(G);
 
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.full);
-  uint64_t* empty = reinterpret_cast<uint64_t*>(sm + L.empty);
-  float* wsw = reinterpret_cast<float*>(sm + L.wsw) + warp * kBlocksPerWarp * G;
+  uint32_t* rel_s = reinterpret_cast<uint32_t*>(sm + L.rel);  // [kStages] warps released, ever
+  volatile uint32_t* abort_s = rel_s + kStages;                // a wait gave up: issue no more
+  uint32_t* issued_s = rel_s + kStages + 1;                    // tiles issued so far
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   float* qn_s = reinterpret_cast<float*>(sm + L.qn);
-  float* comp_s = reinterpret_cast<float*>(sm + L.comp);
   float* refw_s = reinterpret_cast<float*>(sm + L.refw);
   float* red_s = reinterpret_cast<float*>(sm + L.red);
   float* logn_s = reinterpret_cast<float*>(sm + L.logn);
   const uint64_t policy = l2_evict_first_policy();
 
-  // Refills the stage of local tile k (warp 0 only; all 32 lanes).
+  // Refills the stage of local tile k (one whole warp).
   auto issue = [&](int k) {
     const int f = f0 + k;
     const int pr = f / TP, t = f % TP;
@@ -139,101 +132,111 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 32 + 1);
-      mbar_init(&empty[s], kWarps);
+      rel_s[s] = 0;
     }
+    *abort_s = 0;
+    *issued_s = min(nt, kStages);
     mbar_init_fence();
   }
   if (tid < 17) logn_s[tid] = tid > 0 ? logf(static_cast<float>(tid)) : -CUDART_INF_F;
   __syncthreads();
-  int issued = min(nt, kStages);
   if (warp == 0)
-    for (int k = 0; k < issued; ++k) issue(k);
+    for (int k = 0; k < min(nt, kStages); ++k) issue(k);
   pdl_launch_dependents();
 
-  constexpr int LPB = D / 8;            // lanes per block in the dot phase
-  constexpr int BPP = 32 / LPB;         // blocks per warp per pass
-  constexpr int PASSES = kBlocksPerWarp / BPP;
-  constexpr int LPH = LPB / G;          // lanes per head after the transpose-reduce
-  constexpr int LR = D / 4;             // lanes per mean-value row (4 channels per lane)
-  constexpr int RS = 32 / LR;           // mean-value rows per warp step
-  constexpr int NSL = kWarps * BPP * PASSES;  // scalar lanes per head in the CTA
-  static_assert(PASSES <= LPH, "scalar lanes of a block must cover its passes");
-  const int li = lane % LPB, bsub = lane / LPB;
-  // after the transpose-reduce, lane li of a block group holds head li / LPH; the pass-p value is
-  // moved p lanes up, so lane (h * LPH + p) does the scalar work of (pass p, head h)
-  const int my_pass = li % LPH;
-  const bool head_lane = my_pass < PASSES;
-  const int my_h = li / LPH;
-  const int my_bl = my_pass * BPP + bsub;  // block of this scalar lane within the warp's 4
-  const int c4 = lane % LR, rsub = lane / LR;
-  const int slot = (warp * BPP + bsub) * PASSES + my_pass;
+  // Lane map: lane l holds channels [l VW, l VW + VW) of every row for all G heads (a warp-wide
+  // row load is one contiguous 512 or 256 bytes: each mean key and mean value is read from
+  // shared memory once). One transpose-reduce of the 4 blocks x G heads partial dots over the
+  // 32 lanes leaves lane l with the full dot of one (block, head) pair: LPBK lanes per pair.
+  constexpr int VW = D / 32;                // 4 (D = 128) or 2 (D = 64)
+  constexpr int NVAL = kBlocksPerWarp * G;  // partial dots per lane
+  constexpr int LPBK = 32 / NVAL;           // lanes per (block, head) after the reduce
+  static_assert(VW == 2 || VW == 4, "head_dim must be 64 or 128");
+  static_assert(NVAL <= 32, "at most 8 heads per kv-head");
+  const int my_idx = lane / LPBK;           // value index b * G + h this lane ends with
+  const int my_b = my_idx / G, my_h = my_idx % G;
+  const bool rep = (lane % LPBK) == 0;      // one lane per (block, head) writes and is merged
+  const int slot = warp * kBlocksPerWarp + my_b;  // 0..31 per head
 
-  float2 qreg[G][4];
-  float qnr[4];
-  float acc[G][4];
-  float mref[G];
-  float zmax = -CUDART_INF_F, zsum = 0.f, lsum = 0.f;
+  float2 qv[G][VW / 2];   // q_h at this lane's channels
+  float2 acc[G][VW / 2];  // sum w nu at this lane's channels, per head
+  float qnr[4];           // s^2 |q_{my_h, C_g}|^2 (R = 4)
+  float mref[G];          // this warp's reference logit per head
+  float zmax = -CUDART_INF_F, zsum = 0.f, lsum = 0.f;  // this lane's (block, head) partials
   int cur = -1;
+  float* wsw = reinterpret_cast<float*>(sm + L.wsw) + warp * NVAL;  // weights of the warp's pairs
 
-  // Merges the 8 warps' partials of the current segment (pair `cur`) in a fixed order.
-  auto finish_segment = [&]() {
-    if (RS > 1 && compensate) {  // fold the row subsets of each warp (D < 128)
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-#pragma unroll
-          for (int o = LR; o < 32; o <<= 1) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], o);
-    }
+  // Merges the 8 warps' partials of the current segment (pair `cur`) in a fixed order, with the
+  // stage `free_stage` (no copy in flight) as scratch for the warps' weighted mean-value sums.
+  auto finish_segment = [&](int free_stage) {
     if (lane == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) refw_s[warp * G + h] = mref[h];
     }
-    if (head_lane) {
+    if (rep) {
       red_s[(0 * G + my_h) * 32 + slot] = zmax;
       red_s[(1 * G + my_h) * 32 + slot] = zsum;
     }
-    for (int i = tid; i < G * D; i += kThreads) comp_s[i] = 0.f;
     __syncthreads();
-    float M[G], fw[G];
+    float fw[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      M[h] = -CUDART_INF_F;
-      for (int w = 0; w < kWarps; ++w) M[h] = fmaxf(M[h], refw_s[w * G + h]);
-      fw[h] = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - M[h]);
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, refw_s[w * G + h]);
+      fw[h] = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - M);
     }
-    if (head_lane) red_s[(2 * G + my_h) * 32 + slot] = lsum * pick_h<G>(fw, my_h);
+    float fme = fw[0];
+#pragma unroll
+    for (int h = 1; h < G; ++h) fme = (my_h == h) ? fw[h] : fme;
+    if (rep) red_s[(2 * G + my_h) * 32 + slot] = lsum * fme;
+    float* part = reinterpret_cast<float*>(sm + L.stage0 + L.stage_bytes * free_stage);  // [kWarps][G][D]
     if (compensate) {
-      for (int w = 0; w < kWarps; ++w) {
-        if (warp == w && rsub == 0) {
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) comp_s[h * D + c4 * 4 + e] += fw[h] * acc[h][e];
+      for (int h = 0; h < G; ++h) {
+        float* pw = part + (warp * G + h) * D + lane * VW;
+        if constexpr (VW == 4) {
+          reinterpret_cast<float4*>(pw)[0] =
+              make_float4(fw[h] * acc[h][0].x, fw[h] * acc[h][0].y, fw[h] * acc[h][1].x, fw[h] * acc[h][1].y);
+        } else {
+          reinterpret_cast<float2*>(pw)[0] = make_float2(fw[h] * acc[h][0].x, fw[h] * acc[h][0].y);
         }
-        __syncthreads();
       }
-    } else {
-      __syncthreads();
     }
+    __syncthreads();
     const int k = blockIdx.x - static_cast<int>(((static_cast<long long>(cur) * TP + 1) * p.nctas - 1) / F);
     const size_t rec = static_cast<size_t>(cur) * p.slots + k;
-    if (tid < G) {
-      float zm = -CUDART_INF_F, zs = 0.f, ls = 0.f;
-      for (int s = 0; s < NSL; ++s) {
-        lse_merge(zm, zs, red_s[(0 * G + tid) * 32 + s], red_s[(1 * G + tid) * 32 + s]);
-        ls += red_s[(2 * G + tid) * 32 + s];
+    if (warp < G) {  // warp hh: head hh's 32 slots, butterfly merges (fixed order)
+      const int hh = warp;
+      float zm = red_s[(0 * G + hh) * 32 + lane], zs = red_s[(1 * G + hh) * 32 + lane];
+      float ls = red_s[(2 * G + hh) * 32 + lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, zm, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, zs, o);
+        lse_merge(zm, zs, m2, s2);
+        ls += __shfl_xor_sync(0xffffffffu, ls, o);
       }
-      p.zpart[(rec * G + tid) * 2] = zm;
-      p.zpart[(rec * G + tid) * 2 + 1] = zs;
-      if (compensate) {
-        p.comp[(rec * G + tid) * (D + 2)] = pick_h<G>(M, tid);
-        p.comp[(rec * G + tid) * (D + 2) + 1] = ls;
+      if (lane == 0) {
+        p.zpart[(rec * G + hh) * 2] = zm;
+        p.zpart[(rec * G + hh) * 2 + 1] = zs;
+        if (compensate) {
+          float Mh = -CUDART_INF_F;
+          for (int w = 0; w < kWarps; ++w) Mh = fmaxf(Mh, refw_s[w * G + hh]);
+          p.comp[(rec * G + hh) * (D + 2)] = Mh;
+          p.comp[(rec * G + hh) * (D + 2) + 1] = ls;
+        }
       }
     }
-    if (compensate)
-      for (int i = tid; i < G * D; i += kThreads) p.comp[(rec * G + i / D) * (D + 2) + 2 + (i % D)] = comp_s[i];
-    __syncthreads();
+    if (compensate) {
+      for (int i = tid; i < G * D; i += kThreads) {
+        float v = part[i];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) v += part[w * G * D + i];
+        p.comp[(rec * G + i / D) * (D + 2) + 2 + (i % D)] = v;
+      }
+    }
+    __syncthreads();  // the scratch stage and the slots are free again
   };
 
   // Loads the query heads of pair `pr` and resets the running state.
@@ -243,10 +246,10 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     __syncthreads();
     const int gsz = D / r;
     for (int i = tid; i < G * r; i += kThreads) {
-      const int h = i / r, g = i % r;
+      const int hh = i / r, g = i % r;
       float s = 0.f;
-      for (int c = 0; c < gsz; ++c) {
-        const float x = q_s[h * D + g * gsz + c];
+      for (int cc = 0; cc < gsz; ++cc) {
+        const float x = q_s[hh * D + g * gsz + cc];
         s = fmaf(x, x, s);
       }
       qn_s[i] = p.scale * p.scale * s;
@@ -254,12 +257,12 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      qreg[h][0] = make_float2(q_s[h * D + li * 4 + 0], q_s[h * D + li * 4 + 1]);
-      qreg[h][1] = make_float2(q_s[h * D + li * 4 + 2], q_s[h * D + li * 4 + 3]);
-      qreg[h][2] = make_float2(q_s[h * D + D / 2 + li * 4 + 0], q_s[h * D + D / 2 + li * 4 + 1]);
-      qreg[h][3] = make_float2(q_s[h * D + D / 2 + li * 4 + 2], q_s[h * D + D / 2 + li * 4 + 3]);
+      const float* qh = q_s + h * D + lane * VW;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+      for (int e = 0; e < VW / 2; ++e) {
+        qv[h][e] = make_float2(qh[2 * e], qh[2 * e + 1]);
+        acc[h][e] = make_float2(0.f, 0.f);
+      }
       mref[h] = -CUDART_INF_F;
     }
     if constexpr (R == 4) {
@@ -274,35 +277,27 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   // `ok` goes false (for this warp) once a wait gives up; the warp then stops waiting and
   // computing but keeps the loop's structure, so every CTA barrier stays matched.
   bool ok = true;
-  int first_unwaited = nt;
 #pragma unroll 1
   for (int k = 0; k < nt; ++k) {
     const int f = f0 + k;
     const int pr = f / TP;
     if (pr != cur) {  // every warp reaches this at the same tile
       __syncthreads();
-      if (cur >= 0) finish_segment();
+      // the stage of tile k - 1 is free: its refill waits until this segment switch is done
+      if (cur >= 0) finish_segment((k + kStages - 1) % kStages);
       start_segment(pr);
       cur = pr;
-    }
-    const int st = k % kStages;
-    // warp 0 refills the stage of tile k + kStages - 1 once every warp has released tile k - 1
-    if (warp == 0 && k >= 1 && k + kStages - 1 < nt) {
-      const int kk = k + kStages - 1;
-      bool freed = ok && mbar_wait(&empty[kk % kStages], ((kk / kStages) - 1) & 1, p.status);
-      freed = __all_sync(0xffffffffu, freed);
-      if (freed) {
-        issue(kk);
-        ++issued;
-      } else {
-        ok = false;
+      if (warp == 0 && k >= 1 && k + kStages - 1 < nt && *abort_s == 0) {
+        issue(k + kStages - 1);
+        if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(k + kStages));
       }
     }
+    const int st = k % kStages;
     bool got = ok && mbar_wait(&full[st], (k / kStages) & 1, p.status);
     got = __all_sync(0xffffffffu, got);
     if (!got && ok) {
       ok = false;
-      first_unwaited = k;
+      if (lane == 0) *abort_s = 1;
     }
     const int jt0 = (f % TP) * kTile;
     const int tn = ok ? min(kTile, p.Nb - jt0) : 0;
@@ -311,122 +306,159 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     const float* nu_t = reinterpret_cast<const float*>(sb + L.off_nu);
     const float* var_t = reinterpret_cast<const float*>(sb + L.off_var);
     const int* cnt_t = reinterpret_cast<const int*>(sb + L.off_cnt);
+    const int jw = warp * kBlocksPerWarp;  // the warp's first block in the tile
 
-    // ---- (1) dots of this warp's blocks with the G heads
-    float v[PASSES][G];
+    // ---- (1) partial dots over this lane's channels: 4 blocks x G heads
+    float v[NVAL];
 #pragma unroll
-    for (int pass = 0; pass < PASSES; ++pass) {
-      const int jt = warp * kBlocksPerWarp + pass * BPP + bsub;
-      const float4 a = reinterpret_cast<const float4*>(mu_t + jt * D)[li];
-      const float4 b = reinterpret_cast<const float4*>(mu_t + jt * D + D / 2)[li];
+    for (int b = 0; b < kBlocksPerWarp; ++b) {
+      const float* row = mu_t + (jw + b) * D + lane * VW;
+      float2 a[VW / 2];
+      if constexpr (VW == 4) {
+        const float4 a4 = reinterpret_cast<const float4*>(row)[0];
+        a[0] = make_float2(a4.x, a4.y);
+        a[1] = make_float2(a4.z, a4.w);
+      } else {
+        a[0] = reinterpret_cast<const float2*>(row)[0];
+      }
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float2 s2 = __fmul2_rn(qreg[h][0], make_float2(a.x, a.y));
-        s2 = __ffma2_rn(qreg[h][1], make_float2(a.z, a.w), s2);
-        s2 = __ffma2_rn(qreg[h][2], make_float2(b.x, b.y), s2);
-        s2 = __ffma2_rn(qreg[h][3], make_float2(b.z, b.w), s2);
-        v[pass][h] = s2.x + s2.y;
+      for (int hh = 0; hh < G; ++hh) {
+        float2 s2 = __fmul2_rn(qv[hh][0], a[0]);
+        if constexpr (VW == 4) s2 = __ffma2_rn(qv[hh][1], a[1], s2);
+        v[b * G + hh] = s2.x + s2.y;
       }
     }
-#pragma unroll
-    for (int pass = 0; pass < PASSES; ++pass) TransposeReduce<G, LPB / 2>::run(v[pass], li);
-    float dot = v[0][0];
-#pragma unroll
-    for (int pass = 1; pass < PASSES; ++pass) {
-      const float t = __shfl_up_sync(0xffffffffu, v[pass][0], pass);
-      if (my_pass == pass) dot = t;
-    }
+    TransposeReduce<NVAL, 16>::run(v, lane);  // lane now holds pair my_idx's dot in v[0]
 
-    // ---- (2) per (block, head) scalars, one (block, head) per scalar lane
+    // ---- (2) scalars of (block my_b, head my_h)
+    const int jm = jw + my_b;
     float xs = -CUDART_INF_F;
-    bool need = false;
-    {
-      const int jt = warp * kBlocksPerWarp + my_bl;
-      if (head_lane && jt < tn) {
-        const int n = cnt_t[jt];
-        float vh;
-        if constexpr (R == 4) {
-          const float4 vv = reinterpret_cast<const float4*>(var_t)[jt];
-          vh = qnr[0] * vv.x;
-          vh = fmaf(qnr[1], vv.y, vh);
-          vh = fmaf(qnr[2], vv.z, vh);
-          vh = fmaf(qnr[3], vv.w, vh);
+    if (jm < tn) {
+      const int n = cnt_t[jm];
+      float vh;
+      if constexpr (R == 4) {
+        const float4 vv = reinterpret_cast<const float4*>(var_t)[jm];
+        vh = qnr[0] * vv.x;
+        vh = fmaf(qnr[1], vv.y, vh);
+        vh = fmaf(qnr[2], vv.z, vh);
+        vh = fmaf(qnr[3], vv.w, vh);
+      } else {
+        vh = 0.f;
+        for (int g = 0; g < r; ++g) vh = fmaf(qn_s[my_h * r + g], var_t[jm * r + g], vh);
+      }
+      float uu;
+      if (n > 0) {
+        xs = fmaf(p.scale, v[0], logn_s[min(n, 16)]);
+        const float lm = xs + __logf(1.f + 0.5f * vh);
+        uu = (p.mode == COMPKV_MODE_COMPKV) ? lm + __logf(0.5f * vh) : lm;
+        if (lm > zmax) {
+          zsum = zsum * __expf(zmax - lm) + 1.f;
+          zmax = lm;
         } else {
-          vh = 0.f;
-          for (int g = 0; g < r; ++g) vh = fmaf(qn_s[my_h * r + g], var_t[jt * r + g], vh);
+          zsum += __expf(lm - zmax);
         }
-        const float lbar = p.scale * dot;
-        const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jt;
-        float uu;
-        if (n > 0) {
-          xs = lbar + logn_s[min(n, 16)];
-          const float lm = xs + __logf(1.f + 0.5f * vh);
-          uu = (p.mode == COMPKV_MODE_COMPKV) ? lm + __logf(0.5f * vh) : lm;
-          if (lm > zmax) {
-            zsum = zsum * __expf(zmax - lm) + 1.f;
-            zmax = lm;
-          } else {
-            zsum += __expf(lm - zmax);
-          }
-          need = xs > pick_h<G>(mref, my_h) + kRefSlack;
-        } else {
-          uu = __int_as_float(0x7fffffff);  // NaN marks an empty block
-        }
+      } else {
+        uu = __int_as_float(0x7fffffff);  // NaN marks an empty block
+      }
+      if (rep) {
+        const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jm;
         p.u[row * G + my_h] = uu;
         p.xrec[row * XS + my_h] = xs;
         if (my_h == 0) p.xrec[row * XS + G] = __int_as_float(n);
       }
     }
+
+    // ---- (3) compensation weights and acc_h += w_{j,h} nu_j over the warp's 4 blocks
     if (compensate) {
-      if (__any_sync(0xffffffffu, need)) {  // rare: move this warp's reference up
-        float sc_mine = 1.f;
+      const float mme0 = mref[0];
+      float mme = mme0;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float tm = warp_max((head_lane && my_h == h) ? xs : -CUDART_INF_F);
-          const float nm = (tm > mref[h] + kRefSlack) ? tm : mref[h];
-          const float sc = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - nm);
-          acc[h][0] *= sc; acc[h][1] *= sc; acc[h][2] *= sc; acc[h][3] *= sc;
-          if (my_h == h) sc_mine = sc;
-          mref[h] = nm;
+      for (int hh = 1; hh < G; ++hh) mme = (my_h == hh) ? mref[hh] : mme;
+      const bool need = xs > mme + kRefSlack;
+      if (__any_sync(0xffffffffu, need)) {  // rare: move the warp's reference up
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float tm = warp_max((need && my_h == hh) ? xs : -CUDART_INF_F);
+          if (tm > mref[hh] + kRefSlack) {
+            const float sc = (mref[hh] == -CUDART_INF_F) ? 0.f : __expf(mref[hh] - tm);
+            const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+            for (int e = 0; e < VW / 2; ++e) acc[hh][e] = __fmul2_rn(acc[hh][e], sc2);
+            if (my_h == hh) lsum *= sc;
+            mref[hh] = tm;
+          }
         }
-        lsum *= sc_mine;
+        mme = mref[0];
+#pragma unroll
+        for (int hh = 1; hh < G; ++hh) mme = (my_h == hh) ? mref[hh] : mme;
       }
-      if (head_lane) {
-        const float w = (xs == -CUDART_INF_F) ? 0.f : __expf(xs - pick_h<G>(mref, my_h));
-        wsw[my_bl * G + my_h] = w;
-        lsum += w;
-      }
+      const float w = (xs == -CUDART_INF_F) ? 0.f : __expf(xs - mme);
+      lsum += w;
+      if (rep) wsw[my_idx] = w;
       __syncwarp();
-      // ---- (3) acc_h += w_{j,h} nu_j over this warp's blocks: 4 channels x G heads per lane
 #pragma unroll
-      for (int b0 = 0; b0 < kBlocksPerWarp; b0 += RS) {
-        const int bl = b0 + rsub;
-        const int jt = warp * kBlocksPerWarp + bl;
-        if (jt < tn) {
-          const float4 nv = reinterpret_cast<const float4*>(nu_t + jt * D)[c4];
+      for (int b = 0; b < kBlocksPerWarp; ++b) {
+        if (jw + b < tn) {
+          const float* row = nu_t + (jw + b) * D + lane * VW;
+          float2 a[VW / 2];
+          if constexpr (VW == 4) {
+            const float4 a4 = reinterpret_cast<const float4*>(row)[0];
+            a[0] = make_float2(a4.x, a4.y);
+            a[1] = make_float2(a4.z, a4.w);
+          } else {
+            a[0] = reinterpret_cast<const float2*>(row)[0];
+          }
+          float wb[G];
+          if constexpr (G % 4 == 0) {
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float w = wsw[bl * G + h];
-            const float2 w2 = make_float2(w, w);
-            const float2 lo = __ffma2_rn(w2, make_float2(nv.x, nv.y), make_float2(acc[h][0], acc[h][1]));
-            const float2 hi = __ffma2_rn(w2, make_float2(nv.z, nv.w), make_float2(acc[h][2], acc[h][3]));
-            acc[h][0] = lo.x;
-            acc[h][1] = lo.y;
-            acc[h][2] = hi.x;
-            acc[h][3] = hi.y;
+            for (int q4 = 0; q4 < G / 4; ++q4) {
+              const float4 t = reinterpret_cast<const float4*>(wsw + b * G)[q4];
+              wb[4 * q4] = t.x;
+              wb[4 * q4 + 1] = t.y;
+              wb[4 * q4 + 2] = t.z;
+              wb[4 * q4 + 3] = t.w;
+            }
+          } else {
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) wb[hh] = wsw[b * G + hh];
+          }
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float2 w2 = make_float2(wb[hh], wb[hh]);
+#pragma unroll
+            for (int e = 0; e < VW / 2; ++e) acc[hh][e] = __ffma2_rn(w2, a[e], acc[hh][e]);
           }
         }
       }
     }
+
+    // release the stage; the last of the 8 warps to do so refills it with tile k + kStages
+    // (unless tile k + 1 starts a new segment: then the refill waits for the segment switch)
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
-  }
-  if (!ok && warp == 0) {
-    // a wait gave up (status recorded): wait, bounded, for the copies warp 0 issued
-    for (int k = first_unwaited; k < issued; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, nullptr);
+    uint32_t before = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      before = atomicAdd(&rel_s[st], 1u);
+    }
+    before = __shfl_sync(0xffffffffu, before, 0);
+    if (before % kWarps == kWarps - 1) {
+      const int kk = k + kStages;
+      const bool defer = k + 1 < nt && (f + 1) / TP != pr;
+      if (kk < nt && !defer && *abort_s == 0) {
+        fence_proxy_async();
+        issue(kk);
+        if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(kk + 1));
+      }
+    }
   }
   __syncthreads();
-  if (cur >= 0) finish_segment();
+  if (*abort_s != 0 && warp == 0) {
+    // a wait gave up (status recorded): wait, bounded, for the copies still in flight
+    const int n_iss = static_cast<int>(*issued_s);
+    for (int k = max(0, n_iss - kStages); k < n_iss; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, nullptr);
+  }
+  __syncthreads();
+  if (cur >= 0) finish_segment(0);
 }
 
 template <typename TQ, int D, int G>
