@@ -522,4 +522,142 @@ __device__ int cta_select_ordered(KeyAt key_at, int n, const RadixCut& cut, int*
   return kept_total;
 }
 
+
+// Address of `p` (this CTA's shared memory) in the shared memory of cluster rank `rank`, as a
+// shared::cluster address.
+__device__ __forceinline__ uint32_t cluster_smem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+// Arrives on an mbarrier of another CTA of the cluster; release at cluster scope, so this
+// thread's earlier writes (to that CTA's shared memory too) are visible to its waiters.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Bounded wait, with acquire at cluster scope (for arrivals made by other CTAs of the cluster).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int32_t* status) {
+  for (uint32_t it = 0; it < (1u << 22); ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  if (status != nullptr) atomicOr(status, COMPKV_DEVERR_WAIT_TIMEOUT);
+  return false;
+}
+
+// Split cluster barrier (all threads of every CTA of the cluster). An early relaxed arrive and a
+// later wait cost almost nothing; after the wait every CTA of the cluster has started, so its
+// shared memory may be written remotely.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------------ warp-level Top-32
+
+// Selection order as one 64-bit code: higher is better. Score key descending, then block index
+// ascending (ties go to the lower index); every real block's code is nonzero, so 0 pads a list.
+__device__ __forceinline__ uint64_t topk_code(uint32_t key, int idx) {
+  return (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(idx));
+}
+__device__ __forceinline__ int topk_index(uint64_t code) {
+  return static_cast<int>(~static_cast<uint32_t>(code));
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int o) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v), o);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), o);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v), src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), src);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Bitonic sort of one value per lane, descending over the lanes (15 compare-exchange steps).
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint64_t o = shfl_xor_u64(v, j);
+      const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
+      v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  }
+  return v;
+}
+
+// The 32 largest of two descending lists (one entry per lane), descending: the elementwise max
+// of a and reversed b is bitonic and holds them; a half-cleaner cascade sorts it.
+__device__ __forceinline__ uint64_t warp_merge_top32(uint64_t a, uint64_t b) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t br = shfl_u64(b, 31 - lane);
+  uint64_t v = a > br ? a : br;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint64_t o = shfl_xor_u64(v, j);
+    const bool lower = (lane & j) == 0;
+    v = lower ? (v > o ? v : o) : (v < o ? v : o);
+  }
+  return v;
+}
+
+// Ascending bitonic sort of one int per lane.
+__device__ __forceinline__ int warp_sort_asc(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool keep_min = ((lane & k) == 0) == ((lane & j) == 0);
+      v = keep_min ? min(v, o) : max(v, o);
+    }
+  }
+  return v;
+}
+
+// This CTA's 32 best codes of items [0, n) (code_at(i)), descending, in lists[0..31]. Each warp
+// scans a contiguous run in chunks of 32 (sort, merge into its running list); the 8 warp lists
+// then merge pairwise in 3 levels. `lists` needs kWarps * 32 entries. Contains CTA barriers.
+// Merges the 8 warps' descending lists (`best` in each warp) into lists[0..31], pairwise in 3
+// levels. `lists` needs kWarps * 32 entries. Contains CTA barriers.
+__device__ __forceinline__ void cta_merge_warp_lists(uint64_t best, uint64_t* lists) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  lists[warp * 32 + lane] = best;
+  __syncthreads();
+#pragma unroll
+  for (int s = 1; s < kWarps; s <<= 1) {
+    if ((warp & (2 * s - 1)) == 0) best = warp_merge_top32(best, lists[(warp + s) * 32 + lane]);
+    __syncthreads();
+    if ((warp & (2 * s - 1)) == 0) lists[warp * 32 + lane] = best;
+    __syncthreads();
+  }
+}
+
+template <typename CodeAt>
+__device__ void cta_top32(CodeAt code_at, int n, uint64_t* lists) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int span = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int i0 = warp * span, i1 = min(n, i0 + span);
+  uint64_t best = 0;
+  for (int b = i0; b < i1; b += 32) {
+    const int i = b + lane;
+    best = warp_merge_top32(best, warp_sort_desc(i < i1 ? code_at(i) : 0ull));
+  }
+  cta_merge_warp_lists(best, lists);
+}
+
 }  // namespace compkv

@@ -11,20 +11,26 @@
 // One thread-block cluster of C CTAs per (sequence, kv-head); rank c owns the blocks
 // [c*chunk, c*chunk + chunk):
 //  1. log Zhat_h (log-sum-exp over the segments), S_j = sum_h exp(u_{j,h} - log Zhat_h) for the
-//     rank's blocks as order-preserving uint32 keys (empty blocks key 0), and the rank's local
-//     Top-K_b under (S desc, index asc) by radix cut.
-//  2. Rank 0 gathers the C candidate lists over distributed shared memory (ascending block order)
-//     and cuts the global Top-K_b from them; the global Top-K_b under this strict order always
-//     lies inside the union of the local ones, so the result is exact. Meanwhile the other ranks
-//     merge the compensation partials of the kv-head's segments, a slice of channels each.
+//     rank's blocks as order-preserving uint32 keys (empty blocks key 0), and the rank's
+//     candidates: its own best under (S desc, index asc).
+//  2. Rank 0 takes the global Top-K_b from the C candidate lists, read over distributed shared
+//     memory; the global Top-K_b under this strict order always lies inside the union of the
+//     local ones, so the result is exact. For K_b <= 32 the lists are each rank's best 32 as
+//     64-bit codes (key, then index), built and merged with warp bitonic networks; above that,
+//     radix selection. Meanwhile the other ranks merge the compensation partials of the
+//     kv-head's segments, a slice of channels each.
 //  3. Rank c attends the c-th contiguous slice of rank 0's ordered selection (balanced whatever
-//     the blocks' positions): bulk copies of their K and V rows (up to the
+//     the blocks' positions; rank 0 writes each rank's slots into its shared memory and releases
+//     them with a remote mbarrier arrive): bulk copies of their K and V rows (up to the
 //     cache capacity; rows past the block's token count are masked) and of their mean values,
 //     exact logits, an online softmax per head, P.V, and removal of the blocks' compensation terms
 //     (taken against the running max of the exact logits, which is at least every processed
 //     block's mean logit, so nothing overflows; a block's compensation mass never exceeds its
 //     exact mass, so the removal cancels at most what it adds).
-//  4. Rank 0 merges the ranks' partials with the compensation partial.
+//  4. Every rank pushes its partial of each output slice into the rank that merges the slice
+//     (distributed shared memory stores); after one cluster barrier each merging rank combines
+//     its slice from local memory with the compensation partial (with selection, the slice whose
+//     compensation sum it merged).
 // Flags run steps 1-2 only (score/select call) or steps 3-4 only on a given selection (sparse
 // decode call). Launched with programmatic dependent launch: the prologue overlaps the previous
 // kernel's tail.
@@ -44,6 +50,7 @@ namespace {
 constexpr int kMaxCluster = 16;
 constexpr int kRound = 8;  // selected blocks per shared-memory round
 constexpr int kRows = kRound * kBlockTokens;
+constexpr int kWarpTopK = 32;  // K_b up to this: warp bitonic Top-K; above: radix select
 
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
@@ -51,7 +58,7 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast
 struct FLay {
   int chunk, ccap, gcap, slots;
   size_t keys, ck, ci, gk, gi, hist, bc, sh, misc, zm, zs, fm, fl, cslice, selm;
-  size_t q, kbuf, vbuf, nu, lg, pT, red, acc, cp, ml, blk, xr, pw, sc, fac, mbar, total;
+  size_t q, kbuf, vbuf, nu, lg, pT, red, acc, ml, blk, xr, pw, sc, fac, mbar, total;
   __host__ __device__ void build(int chunk_, int Kb, int C, int slots_, int G, int D, int esz, int ksub) {
     chunk = chunk_;
     slots = slots_;
@@ -80,9 +87,8 @@ struct FLay {
     lg = o;     o = a16(o + sizeof(float) * G * kRows);
     pT = o;     o = a16(o + sizeof(float) * G * kRows);
     red = o;    o = a16(o + sizeof(float) * (ksub * G * D > 256 ? ksub * G * D : 256));
-    acc = o;    o = a16(o + sizeof(float) * G * D);
-    cp = o;     o = a16(o + sizeof(float) * G * (D + 2));
-    ml = o;     o = a16(o + sizeof(float) * 16);
+    acc = o;    o = a16(o + sizeof(float) * 2 * G * D);          // received partials [C][slice]
+    ml = o;     o = a16(o + sizeof(float) * kMaxCluster * 2 * G);  // received (m, l) [C][G][2]
     blk = o;    o = a16(o + sizeof(int) * 2 * kRound);
     xr = o;     o = a16(o + sizeof(float) * G * kRound);
     pw = o;     o = a16(o + sizeof(float) * G * kRound);
@@ -160,7 +166,6 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   float* pT = reinterpret_cast<float*>(sm + L.pT);
   float* red = reinterpret_cast<float*>(sm + L.red);
   float* acc_s = reinterpret_cast<float*>(sm + L.acc);
-  float* cp_s = reinterpret_cast<float*>(sm + L.cp);
   float* ml_s = reinterpret_cast<float*>(sm + L.ml);
   int* blk_j = reinterpret_cast<int*>(sm + L.blk);
   int* blk_n = blk_j + kRound;
@@ -172,7 +177,8 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
 
   // ---- prologue (inputs written before the streaming kernel started)
   if (tid == 0) {
-    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[0], 1);  // K/V rows of an attention round
+    mbar_init(&mbar[1], 1);  // this rank's selection slots, delivered by rank 0
     mbar_init_fence();
   }
   if (p.do_attend) {
@@ -183,6 +189,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   const int li = lane % RG::kLpr;
   float qr[G][EPV];
   if (p.do_attend) load_q_regs<T, D, G>(q_s, li, qr);
+  cluster_arrive_relaxed();  // matched by cluster_wait() before this CTA first writes a peer
 
   pdl_wait();  // the previous kernel's outputs are visible from here on
 
@@ -207,13 +214,16 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         fl_s[t] = cs[static_cast<size_t>(t) * (D + 2) + 1];
       }
     }
+    // warp w keys the local blocks [w span, w span + span), 32 at a time (lane-contiguous)
+    const int span = ((nloc + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+    const int jb = warp * span;
     constexpr int UPT = 4;  // log-score rows prefetched per thread before log Zhat is known
     float ur[UPT][G];
 #pragma unroll
     for (int k = 0; k < UPT; ++k) {
-      const int j = tid + k * kThreads;
+      const int j = jb + k * 32 + lane;
 #pragma unroll
-      for (int h = 0; h < G; ++h) ur[k][h] = (j < nloc) ? up[static_cast<size_t>(j) * G + h] : 0.f;
+      for (int h = 0; h < G; ++h) ur[k][h] = (k * 32 < span && j < nloc) ? up[static_cast<size_t>(j) * G + h] : 0.f;
     }
     __syncthreads();
     // ---- 1b. log Zhat per head; compensation max, factors and sum per head
@@ -228,30 +238,16 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         lse_merge(m, s, m2, s2);
       }
       if (lane == 0) logz[h] = (m == -CUDART_INF_F) ? -CUDART_INF_F : m + logf(s);
-      if (compensate) {
-        float M = -CUDART_INF_F;
-        for (int t = lane; t < nseg; t += 32) M = fmaxf(M, fm_s[t * G + h]);
-        M = warp_max(M);
-        float l = 0.f;
-        for (int t = lane; t < nseg; t += 32) {
-          const float mt = fm_s[t * G + h];
-          const float f = (mt == -CUDART_INF_F) ? 0.f : __expf(mt - M);
-          fm_s[t * G + h] = f;
-          l = fmaf(f, fl_s[t * G + h], l);
-        }
-        l = warp_sum(l);
-        if (lane == 0) {
-          cM[h] = M;
-          cl[h] = l;
-        }
-      }
     }
     __syncthreads();
-    // ---- 1c. keys of this rank's blocks
+    // ---- 1c/1d. keys of this rank's blocks and its candidates
     float lz[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) lz[h] = logz[h];
-    for (int k = 0, j = tid; j < nloc; ++k, j += kThreads) {
+    const bool warp_topk = Kb > 0 && Kb <= kWarpTopK;
+    // S_j of chunk k of this warp, as a key (empty blocks: 0); also written to `scores`
+    auto key_of = [&](int k, int j) -> uint32_t {
+      if (j >= nloc) return 0u;
       float S = 0.f;
       if (k < UPT) {
 #pragma unroll
@@ -265,34 +261,113 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         for (int h = 0; h < G; ++h) S += __expf(up[static_cast<size_t>(j) * G + h] - lz[h]);
       }
       const bool empty = S != S;
-      keys[j] = empty ? 0u : score_key(S);
       if (p.scores) p.scores[static_cast<size_t>(pr) * p.Nb + j0 + j] = empty ? 0.f : S;
-    }
-    __syncthreads();
-    // ---- 1d. local Top-K_b candidates, in ascending block order
+      return empty ? 0u : score_key(S);
+    };
     if (tid == 0) misc[0] = 0;
-    if (Kb > 0) {
-      int ncand;
-      if (nloc <= Kb) {
-        for (int j = tid; j < nloc; j += kThreads) {
-          ck[j] = keys[j];
-          ci[j] = j0 + j;
-        }
-        ncand = nloc;
-      } else {
-        auto kat = [&](int i) { return keys[i]; };
-        const RadixCut cut = cta_topk_cut(kat, nloc, Kb, hist, bc, shs);
-        ncand = cta_select_ordered_w(kat, nloc, cut, shs, [&](int i, int pos) {
-          ck[pos] = keys[i];
-          ci[pos] = j0 + i;
-        });
+    if (warp_topk) {
+      // this rank's best 32 (descending codes) in hist[0..255]: a superset of its share. Chunks
+      // go in pairs: two independent sorts, then one merge.
+      uint64_t best = 0ull;
+      for (int k = 0; k * 32 < span; k += 2) {
+        const int ja = jb + k * 32 + lane, jc = ja + 32;
+        const uint32_t ka = key_of(k, ja);
+        const uint32_t kc = ((k + 1) * 32 < span) ? key_of(k + 1, jc) : 0u;
+        const uint64_t sa = warp_sort_desc(ja < nloc ? topk_code(ka, j0 + ja) : 0ull);
+        const uint64_t sc = warp_sort_desc(((k + 1) * 32 < span && jc < nloc) ? topk_code(kc, j0 + jc) : 0ull);
+        const uint64_t m2 = warp_merge_top32(sa, sc);
+        best = (k == 0) ? m2 : warp_merge_top32(best, m2);
       }
-      if (tid == 0) misc[0] = ncand;
+      cta_merge_warp_lists(best, reinterpret_cast<uint64_t*>(hist));
+      if (p.do_attend && warp == 0) {
+        // speculative: this rank's likeliest picks start moving from HBM to L2 while the global
+        // cut runs (about 2 K_b / C of them: the global Top-K_b holds K_b / C per rank on average)
+        const int m = min(32, max(1, (2 * Kb + C - 1) / C));
+        const uint64_t code = reinterpret_cast<const uint64_t*>(hist)[lane];
+        if (lane < m && code != 0ull) {
+          const int j = topk_index(code);
+          const size_t off = (static_cast<size_t>(pr) * p.T + static_cast<size_t>(j) * kBlockTokens) * D;
+          const size_t bytes = static_cast<size_t>(min(kBlockTokens, p.T - j * kBlockTokens)) * D * sizeof(T);
+          prefetch_l2_range(static_cast<const T*>(p.K) + off, bytes);
+          prefetch_l2_range(static_cast<const T*>(p.V) + off, bytes);
+        }
+      }
+    } else {
+      for (int k = 0; k * 32 < span; ++k) {
+        const int j = jb + k * 32 + lane;
+        const uint32_t key = key_of(k, j);
+        if (j < nloc) keys[j] = key;
+      }
+      __syncthreads();
+      if (Kb > 0) {
+        int ncand;
+        if (nloc <= Kb) {
+          for (int j = tid; j < nloc; j += kThreads) {
+            ck[j] = keys[j];
+            ci[j] = j0 + j;
+          }
+          ncand = nloc;
+        } else {
+          auto kat = [&](int i) { return keys[i]; };
+          const RadixCut cut = cta_topk_cut(kat, nloc, Kb, hist, bc, shs);
+          ncand = cta_select_ordered_w(kat, nloc, cut, shs, [&](int i, int pos) {
+            ck[pos] = keys[i];
+            ci[pos] = j0 + i;
+          });
+        }
+        if (tid == 0) misc[0] = ncand;
+      }
+    }
+    cluster_wait();  // every rank has started: peers' shared memory may be written
+    if (warp_topk && warp == 0) {  // push this rank's list to rank 0
+      const uint64_t code = reinterpret_cast<const uint64_t*>(hist)[lane];
+      *cluster.map_shared_rank(reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + rank * 32 + lane, 0) = code;
     }
     cluster.sync();  // #1: every rank's candidates are visible
 
-    // ---- 2. rank 0: global cut over the gathered candidates; other ranks: compensation merge
-    if (rank == 0 && Kb > 0) {
+    // ---- 2. rank 0: global Top-K_b from the ranks' candidates; other ranks: compensation merge
+    if (rank == 0 && Kb > 0 && Kb <= kWarpTopK) {
+      // merge the C ranks' best-32 lists pairwise (the first level straight from the ranks'
+      // shared memory), then order the first K_b by block index
+      const uint64_t* rl = reinterpret_cast<const uint64_t*>(hist) + kWarps * 32;  // [C][32] pushed
+      uint64_t* g0 = reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + kMaxCluster * 32;
+      uint64_t* g1 = g0 + kWarps * 32;
+      int nl = 1;
+      if (C == 1) {
+        if (warp == 0) g0[lane] = rl[lane];
+      } else {
+        if (warp < C / 2) g0[warp * 32 + lane] = warp_merge_top32(rl[2 * warp * 32 + lane], rl[(2 * warp + 1) * 32 + lane]);
+        nl = C / 2;
+      }
+      __syncthreads();
+      uint64_t* src = g0;
+      uint64_t* dst = g1;
+      while (nl > 1) {
+        if (warp < nl / 2)
+          dst[warp * 32 + lane] = warp_merge_top32(src[2 * warp * 32 + lane], src[(2 * warp + 1) * 32 + lane]);
+        __syncthreads();
+        uint64_t* t = src;
+        src = dst;
+        dst = t;
+        nl /= 2;
+      }
+      if (warp == 0) {
+        const int idx = warp_sort_asc(lane < Kb ? topk_index(src[lane]) : 0x7fffffff);
+        if (lane < Kb && p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + lane] = idx;
+        if (p.do_attend) {
+          // lane r writes rank r's slots [r per, r per + per) into its shared memory, then
+          // releases them to it with a remote arrive: rank r starts at once, no cluster barrier
+          const int per = (Kb + C - 1) / C;
+          for (int q = 0; q < per; ++q) {
+            const int slot = lane * per + q;
+            const int v = __shfl_sync(0xffffffffu, idx, slot < 32 ? slot : 0);
+            if (lane < C && slot < Kb) *cluster.map_shared_rank(&selm[q], lane) = v;
+          }
+          if (lane < C) mbar_arrive_remote(cluster_smem_addr(&mbar[1], lane));
+        }
+        if (lane == 0) misc[6] = Kb;
+      }
+    } else if (rank == 0 && Kb > 0) {
       if (tid < C) misc[24 + tid] = *cluster.map_shared_rank(&misc[0], tid);
       __syncthreads();
       if (tid == 0) {
@@ -326,6 +401,26 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       if (tid == 0) misc[6] = nout;
     }
     if (compensate && (C == 1 || rank != 0)) {
+      // compensation reference, segment factors and sum per head (off the selection's path)
+      if (warp < G) {
+        const int h = warp;
+        float M = -CUDART_INF_F;
+        for (int t = lane; t < nseg; t += 32) M = fmaxf(M, fm_s[t * G + h]);
+        M = warp_max(M);
+        float l = 0.f;
+        for (int t = lane; t < nseg; t += 32) {
+          const float mt = fm_s[t * G + h];
+          const float f = (mt == -CUDART_INF_F) ? 0.f : __expf(mt - M);
+          fm_s[t * G + h] = f;
+          l = fmaf(f, fl_s[t * G + h], l);
+        }
+        l = warp_sum(l);
+        if (lane == 0) {
+          cM[h] = M;
+          cl[h] = l;
+        }
+      }
+      __syncthreads();
       // merge a slice of the compensation partials' channels: lanes along channels (coalesced),
       // 4 segment groups summed in a fixed order
       const int E = G * D, W = (C == 1) ? 1 : C - 1, wr = (C == 1) ? 0 : rank - 1;
@@ -353,15 +448,19 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         __syncthreads();
       }
     }
-    if (compensate && !p.do_attend && rank == 0 && tid < G) {
+    if (compensate && !p.do_attend && rank == (C == 1 ? 0 : 1) && tid < G) {
       float* o = p.comp + (static_cast<size_t>(pr) * G + tid) * (D + 2);
       o[0] = cM[tid];
       o[1] = cl[tid];
     }
-    cluster.sync();  // #2: the cut and the merged compensation slices are visible
+    if (!warp_topk) cluster.sync();  // #2: the cut is visible (radix path; the warp path
+                                      // delivers the slots through mbar[1])
 
     // ---- 3a. this rank's share of the selection: a contiguous slice of rank 0's ordered list
-    if (p.do_attend && Kb > 0) {
+    if (p.do_attend && warp_topk) {  // rank 0 delivers this rank's slots
+      const int per = (Kb + C - 1) / C;
+      nsel = mbar_wait_cluster(&mbar[1], 0, p.status) ? max(0, min(per, Kb - rank * per)) : 0;
+    } else if (p.do_attend && Kb > 0) {
       const int total = *cluster.map_shared_rank(&misc[6], 0);
       const int per = (total + C - 1) / C;
       const int s0 = min(total, rank * per), s1 = min(total, s0 + per);
@@ -379,25 +478,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     nsel = s1 - s0;
     __syncthreads();
   }
-  if (!p.do_attend) return;  // select only: no shared memory of another rank is read after #2
-
-  // compensation partial for the final merge (rank 0), fetched while the attention runs
-  if (rank == 0 && compensate) {
-    if (p.do_select) {
-      const int E = G * D, W = (C == 1) ? 1 : C - 1, per = (E + W - 1) / W;
-      for (int e = tid; e < E; e += kThreads) {
-        const int owner = (C == 1) ? 0 : 1 + e / per;
-        cp_s[(e / D) * (D + 2) + 2 + (e % D)] = *cluster.map_shared_rank(&cslice[e], owner);
-      }
-      if (tid < G) {
-        cp_s[tid * (D + 2)] = cM[tid];
-        cp_s[tid * (D + 2) + 1] = cl[tid];
-      }
-    } else {
-      const float* cp = p.comp + static_cast<size_t>(pr) * G * (D + 2);
-      for (int i = tid; i < G * (D + 2); i += kThreads) cp_s[i] = cp[i];
-    }
-  }
+  if (!p.do_attend) return;  // select only: no rank touches another's shared memory from here
 
   // ---- 3b. exact attention over this rank's selected blocks, in rounds of kRound blocks
   const T* Kbase = static_cast<const T*>(p.K) + static_cast<size_t>(pr) * p.T * D;
@@ -516,68 +597,77 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     __syncthreads();  // buffers are reused by the next round
   }
 
-  // ---- this rank's partial (m, l, acc) per head -> shared memory
+  // ---- this rank's partial (m, l, acc) per head, pushed to the ranks that merge the outputs.
+  // Output channels [0, E) are cut into slices, one per merging rank: with selection ranks
+  // 1..C-1 (each holds the compensation sum of its slice), without it ranks 0..C-1 (C = 1: rank
+  // 0 alone). Every rank writes its partial of a slice into the merging rank's receive buffer.
+  constexpr int E = G * D;
+  const int first_owner = (p.do_select && C > 1) ? 1 : 0;
+  const int n_owners = C - first_owner;
+  const int per_o = (E + n_owners - 1) / n_owners;
+  float* racc = acc_s;  // [C][per_o] received partial sums
+  float* rml = ml_s;    // [C][G][2] received (m, l)
+  if (!p.do_select) cluster_wait();  // every rank has started: peers may be written
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < VEC; ++e) red[(sub * G + h) * D + cv * VEC + e] = acc[h][e];
-  if (warp < G && lane == 0) {
-    ml_s[2 * warp] = m_run;
-    ml_s[2 * warp + 1] = l_run;
+  if (warp < G) {  // (m, l) of head `warp` to every merging rank whose slice touches the head
+    const int h = warp;
+    const int o_lo = first_owner + (h * D) / per_o, o_hi = first_owner + (h * D + D - 1) / per_o;
+    const int o = o_lo + lane;
+    if (o <= o_hi) {
+      float* dst = cluster.map_shared_rank(rml + (rank * G + h) * 2, o);
+      dst[0] = m_run;
+      dst[1] = l_run;
+    }
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += kThreads) {
+  for (int i = tid; i < E; i += kThreads) {
     float sum = 0.f;
-    for (int k = 0; k < PVt::kSub; ++k) sum += red[k * G * D + i];
-    acc_s[i] = sum;
+    for (int k = 0; k < PVt::kSub; ++k) sum += red[k * E + i];
+    const int ow = i / per_o;
+    *cluster.map_shared_rank(racc + rank * per_o + (i - ow * per_o), first_owner + ow) = sum;
   }
-  cluster.sync();  // #3: every rank's partial is visible
+  cluster.sync();  // #3: every partial pushed to this rank is visible
 
-  // ---- 4. rank 0 merges the ranks' partials and the compensation partial
-  if (rank == 0) {
-    if (tid < G * C) {
-      const int h = tid / C, s2 = tid % C;
-      const float* rml = cluster.map_shared_rank(ml_s, s2);
-      fac_s[h * 17 + s2] = rml[2 * h];
-      fac_s[G * 17 + h * 17 + s2] = rml[2 * h + 1];
-    }
-    __syncthreads();
-    if (tid < G) {
-      const int h = tid;
-      const float cmh = compensate ? cp_s[h * (D + 2)] : -CUDART_INF_F;
-      float M = cmh;
-      for (int s2 = 0; s2 < C; ++s2) M = fmaxf(M, fac_s[h * 17 + s2]);
-      float den = 0.f;
-      if (cmh != -CUDART_INF_F) {
-        const float f = __expf(cmh - M);
-        fac_s[h * 17 + 16] = f;
-        den = f * cp_s[h * (D + 2) + 1];
-      } else {
-        fac_s[h * 17 + 16] = 0.f;
-      }
-      for (int s2 = 0; s2 < C; ++s2) {
-        const float ms = fac_s[h * 17 + s2];
+  // ---- 4. outputs of this rank's slice, from its receive buffers (local reads only)
+  const int wr = rank - first_owner;
+  if (wr >= 0) {
+    const int e0 = min(E, wr * per_o), e1 = min(E, e0 + per_o);
+    const float* cpg = p.comp + static_cast<size_t>(pr) * G * (D + 2);
+    if (e0 < e1) {
+      const int hlo = e0 / D, nh = (e1 - 1) / D - hlo + 1;
+      if (warp < nh) {  // warp w: head hlo + w's factors over the C ranks and the compensation
+        const int h = hlo + warp;
+        float cmh = -CUDART_INF_F, clh = 0.f;
+        if (compensate) {
+          cmh = p.do_select ? cM[h] : cpg[h * (D + 2)];
+          clh = p.do_select ? cl[h] : cpg[h * (D + 2) + 1];
+        }
+        const float ms = lane < C ? rml[(lane * G + h) * 2] : -CUDART_INF_F;
+        const float ls = lane < C ? rml[(lane * G + h) * 2 + 1] : 0.f;
+        const float M = fmaxf(warp_max(ms), cmh);
         const float f = (ms == -CUDART_INF_F) ? 0.f : __expf(ms - M);
-        fac_s[h * 17 + s2] = f;
-        den = fmaf(f, fac_s[G * 17 + h * 17 + s2], den);
+        const float fc = (cmh == -CUDART_INF_F) ? 0.f : __expf(cmh - M);
+        const float den = fmaf(fc, clh, warp_sum(f * ls));
+        if (lane < C) fac_s[warp * 17 + lane] = f;
+        if (lane == 0) {
+          fac_s[warp * 17 + 16] = fc;
+          sc_s[warp] = den > 0.f ? 1.f / den : 0.f;
+        }
       }
-      sc_s[h] = den > 0.f ? 1.f / den : 0.f;
-    }
-    __syncthreads();
-    float* o = p.out + static_cast<size_t>(pr) * G * D;
-    for (int i = tid; i < G * D; i += kThreads) {
-      const int h = i / D, c = i % D;
-      float part[kMaxCluster];
-#pragma unroll
-      for (int s2 = 0; s2 < kMaxCluster; ++s2) part[s2] = (s2 < C) ? cluster.map_shared_rank(acc_s, s2)[i] : 0.f;
-      float a = compensate ? fac_s[h * 17 + 16] * cp_s[h * (D + 2) + 2 + c] : 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < kMaxCluster; ++s2)
-        if (s2 < C) a = fmaf(fac_s[h * 17 + s2], part[s2], a);  // factors past C are not set
-      o[i] = a * sc_s[h];
+      __syncthreads();
+      float* o = p.out + static_cast<size_t>(pr) * E;
+      for (int i = e0 + tid; i < e1; i += kThreads) {
+        const int hs = i / D - hlo, c = i % D;
+        float a = 0.f;
+        if (compensate) a = fac_s[hs * 17 + 16] * (p.do_select ? cslice[i] : cpg[(hs + hlo) * (D + 2) + 2 + c]);
+        for (int s2 = 0; s2 < C; ++s2) a = fmaf(fac_s[hs * 17 + s2], racc[s2 * per_o + (i - e0)], a);
+        o[i] = a * sc_s[hs];
+      }
     }
   }
-  cluster.sync();  // #4: rank 0 is done reading the other ranks' shared memory
 }
 
 template <typename T, int D>

@@ -333,6 +333,8 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     // ---- (2) scalars of (block my_b, head my_h)
     const int jm = jw + my_b;
     float xs = -CUDART_INF_F;
+    float st_u = 0.f;  // stored after the stage is released (the release fence then has no
+    int st_n = 0;      // global stores of this tile to wait for)
     if (jm < tn) {
       const int n = cnt_t[jm];
       float vh;
@@ -360,12 +362,8 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       } else {
         uu = __int_as_float(0x7fffffff);  // NaN marks an empty block
       }
-      if (rep) {
-        const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jm;
-        p.u[row * G + my_h] = uu;
-        p.xrec[row * XS + my_h] = xs;
-        if (my_h == 0) p.xrec[row * XS + G] = __int_as_float(n);
-      }
+      st_u = uu;
+      st_n = n;
     }
 
     // ---- (3) compensation weights and acc_h += w_{j,h} nu_j over the warp's 4 blocks
@@ -449,6 +447,12 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
         issue(kk);
         if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(kk + 1));
       }
+    }
+    if (rep && jm < tn) {
+      const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jm;
+      p.u[row * G + my_h] = st_u;
+      p.xrec[row * XS + my_h] = xs;
+      if (my_h == 0) p.xrec[row * XS + G] = __int_as_float(st_n);
     }
   }
   __syncthreads();
