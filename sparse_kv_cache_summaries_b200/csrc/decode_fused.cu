@@ -120,6 +120,40 @@ struct FParams {
   int32_t* status;
 };
 
+// One lane's part of a K or V row: VEP consecutive elements as one vector load (read-only path).
+template <int BYTES> struct RawOf;
+template <> struct RawOf<4> { using type = uint32_t; };
+template <> struct RawOf<8> { using type = uint2; };
+template <> struct RawOf<16> { using type = uint4; };
+
+template <typename T, int VEP>
+struct RowPart {
+  using Raw = typename RawOf<VEP * static_cast<int>(sizeof(T))>::type;
+  static __device__ __forceinline__ Raw load(const T* row, int lane) {
+    return __ldg(reinterpret_cast<const Raw*>(row) + lane);
+  }
+  static __device__ __forceinline__ Raw zero() {
+    Raw z;
+    uint32_t* u = reinterpret_cast<uint32_t*>(&z);
+#pragma unroll
+    for (int i = 0; i < static_cast<int>(sizeof(Raw)) / 4; ++i) u[i] = 0u;
+    return z;
+  }
+  static __device__ __forceinline__ void unpack(const Raw& w, float (&f)[VEP]) {
+    const uint32_t* u = reinterpret_cast<const uint32_t*>(&w);
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int i = 0; i < VEP / 2; ++i) {
+        f[2 * i] = __uint_as_float(u[i] << 16);
+        f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < VEP; ++i) f[i] = __uint_as_float(u[i]);
+    }
+  }
+};
+
 __device__ __forceinline__ int stream_cta_of_tile(long long f, int nctas, int F) {
   return static_cast<int>(((f + 1) * nctas - 1) / F);
 }
@@ -127,9 +161,6 @@ __device__ __forceinline__ int stream_cta_of_tile(long long f, int nctas, int F)
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_constant__ FParams p) {
-  using RG = RowGeom<T, D>;
-  using PVt = PV<T, D, G>;
-  constexpr int EPV = RG::kEpv, VEC = PVt::kVec;
   constexpr int XS = xrec_stride(G);
   extern __shared__ __align__(128) unsigned char sm[];
   const FLay& L = p.L;
@@ -160,24 +191,16 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   int* selm = reinterpret_cast<int*>(sm + L.selm);
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   T* kbuf = reinterpret_cast<T*>(sm + L.kbuf);
-  T* vbuf = reinterpret_cast<T*>(sm + L.vbuf);
-  float* nu_s = reinterpret_cast<float*>(sm + L.nu);
-  float* lg = reinterpret_cast<float*>(sm + L.lg);
-  float* pT = reinterpret_cast<float*>(sm + L.pT);
+  float* lg_s = reinterpret_cast<float*>(sm + L.lg);
   float* red = reinterpret_cast<float*>(sm + L.red);
   float* acc_s = reinterpret_cast<float*>(sm + L.acc);
   float* ml_s = reinterpret_cast<float*>(sm + L.ml);
-  int* blk_j = reinterpret_cast<int*>(sm + L.blk);
-  int* blk_n = blk_j + kRound;
-  float* xr_s = reinterpret_cast<float*>(sm + L.xr);
-  float* pw_s = reinterpret_cast<float*>(sm + L.pw);
   float* sc_s = reinterpret_cast<float*>(sm + L.sc);
   float* fac_s = reinterpret_cast<float*>(sm + L.fac);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L.mbar);
 
   // ---- prologue (inputs written before the streaming kernel started)
   if (tid == 0) {
-    mbar_init(&mbar[0], 1);  // K/V rows of an attention round
     mbar_init(&mbar[1], 1);  // this rank's selection slots, delivered by rank 0
     mbar_init_fence();
   }
@@ -186,9 +209,6 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     for (int i = tid; i < G * D; i += kThreads) q_s[i] = to_float(qp[i]);
   }
   __syncthreads();
-  const int li = lane % RG::kLpr;
-  float qr[G][EPV];
-  if (p.do_attend) load_q_regs<T, D, G>(q_s, li, qr);
   cluster_arrive_relaxed();  // matched by cluster_wait() before this CTA first writes a peer
 
   pdl_wait();  // the previous kernel's outputs are visible from here on
@@ -480,154 +500,191 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   }
   if (!p.do_attend) return;  // select only: no rank touches another's shared memory from here
 
-  // ---- 3b. exact attention over this rank's selected blocks, in rounds of kRound blocks
+  // ---- 3b. exact attention over this rank's selected blocks. Work unit: a group of 4 rows of
+  // one block; warp w takes groups w, w + 8, ... Each lane holds VEP = D / 32 channels of every
+  // row, read straight into registers (one vector load per row; no shared-memory staging, no
+  // CTA barrier), with an online softmax per warp and head. The group of a block's first rows
+  // also removes the block's compensation term, taken against a reference raised to at least
+  // its mean logit, so no weight exceeds 1.
+  constexpr int VEP = D / 32;
+  constexpr int GR = 4;                      // rows per group
+  constexpr int GPB = kBlockTokens / GR;     // groups per block
+  constexpr int NV = GR * G;                 // (row, head) logits of a group
+  constexpr int LPV = 32 / NV;               // lanes per (row, head) after the reduce
+  static_assert(NV <= 32 && VEP >= 2, "unsupported head layout");
+  using RP = RowPart<T, VEP>;
   const T* Kbase = static_cast<const T*>(p.K) + static_cast<size_t>(pr) * p.T * D;
   const T* Vbase = static_cast<const T*>(p.V) + static_cast<size_t>(pr) * p.T * D;
   const float* NUbase = p.mean_v + static_cast<size_t>(pr) * p.Nb * D;
   const float* XRbase = p.xrec + static_cast<size_t>(pr) * p.Nb * XS;
-  const int cv = tid % PVt::kCols, sub = tid / PVt::kCols;
-  float acc[G][VEC];
+  float qv[G][VEP];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
-  float m_run = -CUDART_INF_F, l_run = 0.f;  // warp h's running state for head h
-  uint32_t phase = 0;
+    for (int e = 0; e < VEP; ++e) qv[h][e] = q_s[h * D + lane * VEP + e];
+  float acc[G][VEP], mw[G], lw[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    mw[h] = -CUDART_INF_F;
+    lw[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < VEP; ++e) acc[h][e] = 0.f;
+  }
+  const int my_v = lane / LPV, my_r = my_v / G, my_h = my_v % G;
+  const int ngroups = nsel * GPB;
 #pragma unroll 1
-  for (int rs0 = 0; rs0 < nsel; rs0 += kRound) {
-    const int nr = min(kRound, nsel - rs0);
-    if (tid < kRound) {
-      int j = (tid < nr) ? selm[rs0 + tid] : -1;
-      if (j < 0 || j >= p.Nb) j = -1;
-      blk_j[tid] = j;
+  for (int g = warp; g < ngroups; g += kWarps) {
+    const int s2 = g / GPB, t0 = (g % GPB) * GR;
+    int j = selm[s2];
+    if (j < 0 || j >= p.Nb) j = -1;
+    const bool first = (g % GPB) == 0;  // this group removes the block's compensation term
+    // loads: the rows up to the cache capacity, the record, and the mean value (first group)
+    typename RP::Raw kr[GR], vr[GR];
+    const int cap = (j >= 0) ? min(kBlockTokens, p.T - j * kBlockTokens) : 0;
+#pragma unroll
+    for (int r = 0; r < GR; ++r) {
+      const bool in = t0 + r < cap;
+      const size_t row = (static_cast<size_t>(j) * kBlockTokens + t0 + r) * D;
+      kr[r] = in ? RP::load(Kbase + row, lane) : RP::zero();
+      vr[r] = in ? RP::load(Vbase + row, lane) : RP::zero();
     }
-    __syncthreads();
-    if (tid == 0) {  // K and V rows up to the cache capacity; the token count comes with the record
-      uint32_t bytes = 0;
-      for (int s2 = 0; s2 < nr; ++s2) {
-        const int j = blk_j[s2];
-        if (j < 0) continue;
-        const int rows = min(kBlockTokens, p.T - j * kBlockTokens);
-        bytes += 2u * rows * D * sizeof(T) + (compensate ? D * sizeof(float) : 0u);
+    const float* rec = XRbase + static_cast<size_t>(j >= 0 ? j : 0) * XS;
+    const int n = (j >= 0) ? max(0, min(__float_as_int(__ldg(rec + G)), cap)) : 0;
+    float xh = -CUDART_INF_F;
+    float nu[VEP];
+#pragma unroll
+    for (int e = 0; e < VEP; ++e) nu[e] = 0.f;
+    if (compensate && first && j >= 0) {
+      xh = __ldg(rec + my_h);
+      const float* nrow = NUbase + static_cast<size_t>(j) * D + lane * VEP;
+#pragma unroll
+      for (int e = 0; e < VEP; ++e) nu[e] = __ldg(nrow + e);
+    }
+    // logits: partial dots over this lane's channels, one transpose-reduce for the group
+    float v[NV];
+    float vf[GR][VEP];
+#pragma unroll
+    for (int r = 0; r < GR; ++r) {
+      float kf[VEP];
+      RP::unpack(kr[r], kf);
+      RP::unpack(vr[r], vf[r]);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float sdot = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEP; ++e) sdot = fmaf(qv[h][e], kf[e], sdot);
+        v[r * G + h] = sdot;
       }
-      mbar_arrive_expect_tx(&mbar[0], bytes);
-      for (int s2 = 0; s2 < nr; ++s2) {
-        const int j = blk_j[s2];
-        if (j < 0) continue;
-        const int rows = min(kBlockTokens, p.T - j * kBlockTokens);
-        const size_t off = static_cast<size_t>(j) * kBlockTokens * D;
-        bulk_g2s(kbuf + s2 * kBlockTokens * D, Kbase + off, rows * D * sizeof(T), &mbar[0]);
-        bulk_g2s(vbuf + s2 * kBlockTokens * D, Vbase + off, rows * D * sizeof(T), &mbar[0]);
-        if (compensate) bulk_g2s(nu_s + s2 * D, NUbase + static_cast<size_t>(j) * D, D * sizeof(float), &mbar[0]);
+    }
+    TransposeReduce<NV, 16>::run(v, lane);  // lane holds (row my_r, head my_h)
+    const bool live = t0 + my_r < n;
+    const float lg = live ? p.scale * v[0] : -CUDART_INF_F;
+    // zero the V parts of rows past the token count (their weight is 0, but 0 * NaN is NaN)
+#pragma unroll
+    for (int r = 0; r < GR; ++r)
+      if (t0 + r >= n) {
+#pragma unroll
+        for (int e = 0; e < VEP; ++e) vf[r][e] = 0.f;
       }
-    }
-    if (tid < nr * (G + 1)) {  // records: x_h and the token count of each block
-      const int s2 = tid / (G + 1), e = tid % (G + 1);
-      const int j = blk_j[s2];
-      const float v = (j >= 0) ? XRbase[static_cast<size_t>(j) * XS + e] : 0.f;
-      if (e < G) xr_s[s2 * G + e] = (j >= 0) ? v : -CUDART_INF_F;
-      else blk_n[s2] = (j >= 0) ? max(0, min(__float_as_int(v), min(kBlockTokens, p.T - j * kBlockTokens))) : 0;
-    }
-    if (tid >= nr && tid < kRound) blk_n[tid] = 0;
-    const bool got = mbar_wait(&mbar[0], phase, p.status);
-    __syncthreads();  // records visible
-    for (int s2 = 0; s2 < nr; ++s2) {  // V rows past a block's token count: zero (0 * NaN is NaN)
-      const int n = blk_n[s2];
-      if (n < kBlockTokens) {
-        T* vrow = vbuf + (static_cast<size_t>(s2) * kBlockTokens + n) * D;
-        for (int e = tid; e < (kBlockTokens - n) * D; e += kThreads) vrow[e] = T(0);
-      }
-    }
-    fence_proxy_async();  // the next round's copies may land on these rows
-    if (__syncthreads_and(got) == 0) {  // uniform: drain (bounded) and stop
-      mbar_wait(&mbar[0], phase, nullptr);
-      break;
-    }
-    phase ^= 1;
-    const int R = nr * kBlockTokens;
-    const int Rpad = (R + kWarps * RG::kRpl - 1) / (kWarps * RG::kRpl) * (kWarps * RG::kRpl);
-    tile_logits<T, D, G>(kbuf, Rpad, qr, p.scale, lg, kRows, [&](int row) {
-      return row < R && (row % kBlockTokens) < blk_n[row / kBlockTokens];
-    });
-    __syncthreads();
-    if (warp < G) {  // softmax update for head h; compensation terms of these blocks removed
-      const int h = warp;
-      float mx = -CUDART_INF_F;
-      for (int row = lane; row < R; row += 32) mx = fmaxf(mx, lg[h * kRows + row]);
-      mx = warp_max(mx);
-      const float m_new = fmaxf(m_run, mx);
-      float ls = 0.f;
-      for (int row = lane; row < R; row += 32) {
-        const float x = lg[h * kRows + row];
-        const float w = (x == -CUDART_INF_F) ? 0.f : __expf(x - m_new);
-        pT[row * G + h] = w;
-        ls += w;
-      }
-      ls = warp_sum(ls);
-      float pw = 0.f;
-      if (compensate && lane < nr) {
-        const float xj = xr_s[lane * G + h];
-        pw = (xj == -CUDART_INF_F) ? 0.f : __expf(xj - m_new);
-      }
-      if (lane < kRound) pw_s[h * kRound + lane] = pw;
-      const float pws = warp_sum(pw);
-      const float scl = (m_run == -CUDART_INF_F) ? 0.f : __expf(m_run - m_new);
-      l_run = l_run * scl + ls - pws;
-      m_run = m_new;
-      if (lane == 0) sc_s[h] = scl;
-    }
-    __syncthreads();
+    // group max per head (over the rows), raised to the removed block's record if any
+    float gm = lg;
+#pragma unroll
+    for (int o = LPV * G; o < 32; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+    gm = fmaxf(gm, xh);
+    float mn[G], sc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float scl = sc_s[h];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[h][e] *= scl;
+      const float gh = __shfl_sync(0xffffffffu, gm, h * LPV);
+      mn[h] = fmaxf(mw[h], gh);
+      sc[h] = (mw[h] == -CUDART_INF_F) ? 0.f : __expf(mw[h] - mn[h]);
     }
-    PVt::accumulate(vbuf, pT, R, sub, cv, acc);
-    if (compensate && sub == 0) {
-      for (int s2 = 0; s2 < nr; ++s2) {
+    float mme = mn[0];
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const float nv = nu_s[s2 * D + cv * VEC + e];
+    for (int h = 1; h < G; ++h) mme = (my_h == h) ? mn[h] : mme;
+    const float pe = (lg == -CUDART_INF_F) ? 0.f : __expf(lg - mme);
+    float ps = pe;
 #pragma unroll
-          for (int h = 0; h < G; ++h) acc[h][e] = fmaf(-pw_s[h * kRound + s2], nv, acc[h][e]);
-        }
+    for (int o = LPV * G; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    const float pw = (xh == -CUDART_INF_F) ? 0.f : __expf(xh - mme);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float psum = __shfl_sync(0xffffffffu, ps, h * LPV);
+      const float pwh = __shfl_sync(0xffffffffu, pw, h * LPV);
+      lw[h] = lw[h] * sc[h] + psum - pwh;
+      mw[h] = mn[h];
+#pragma unroll
+      for (int e = 0; e < VEP; ++e) acc[h][e] = fmaf(-pwh, nu[e], acc[h][e] * sc[h]);
+#pragma unroll
+      for (int r = 0; r < GR; ++r) {
+        const float prh = __shfl_sync(0xffffffffu, pe, (r * G + h) * LPV);
+#pragma unroll
+        for (int e = 0; e < VEP; ++e) acc[h][e] = fmaf(prh, vf[r][e], acc[h][e]);
       }
     }
-    __syncthreads();  // buffers are reused by the next round
   }
 
-  // ---- this rank's partial (m, l, acc) per head, pushed to the ranks that merge the outputs.
-  // Output channels [0, E) are cut into slices, one per merging rank: with selection ranks
-  // 1..C-1 (each holds the compensation sum of its slice), without it ranks 0..C-1 (C = 1: rank
-  // 0 alone). Every rank writes its partial of a slice into the merging rank's receive buffer.
+  // ---- the warps' partials -> this rank's partial (M_h, L_h, A_h) in shared memory
+  float* wacc = reinterpret_cast<float*>(kbuf);  // [kWarps][G][D]
+  float* wml = lg_s;                             // [kWarps][G][2], then factors [kWarps][G]
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int e = 0; e < VEP; ++e) wacc[(warp * G + h) * D + lane * VEP + e] = acc[h][e];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      wml[(warp * G + h) * 2] = mw[h];
+      wml[(warp * G + h) * 2 + 1] = lw[h];
+    }
+  }
+  __syncthreads();
+  float* wf = wml + kWarps * G * 2;  // [kWarps][G] factors
+  float* rM = wf + kWarps * G;       // [G] this rank's reference per head
+  float* rL = rM + G;                // [G]
+  if (tid < G) {
+    const int h = tid;
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wml[(w * G + h) * 2]);
+    float Lsum = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float mwv = wml[(w * G + h) * 2];
+      const float f = (mwv == -CUDART_INF_F) ? 0.f : __expf(mwv - M);
+      wf[w * G + h] = f;
+      Lsum = fmaf(f, wml[(w * G + h) * 2 + 1], Lsum);
+    }
+    rM[h] = M;
+    rL[h] = Lsum;
+  }
+  __syncthreads();
+  // ---- this rank's partial, pushed to the ranks that merge the outputs. Output channels
+  // [0, E) are cut into slices, one per merging rank: with selection ranks 1..C-1 (each holds
+  // the compensation sum of its slice), without it ranks 0..C-1 (C = 1: rank 0 alone). Every
+  // rank writes its partial of a slice into the merging rank's receive buffers.
   constexpr int E = G * D;
   const int first_owner = (p.do_select && C > 1) ? 1 : 0;
   const int n_owners = C - first_owner;
   const int per_o = (E + n_owners - 1) / n_owners;
   float* racc = acc_s;  // [C][per_o] received partial sums
-  float* rml = ml_s;    // [C][G][2] received (m, l)
+  float* rml = ml_s;    // [C][G][2] received (M, L)
   if (!p.do_select) cluster_wait();  // every rank has started: peers may be written
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) red[(sub * G + h) * D + cv * VEC + e] = acc[h][e];
-  if (warp < G) {  // (m, l) of head `warp` to every merging rank whose slice touches the head
+  if (warp < G) {  // (M, L) of head `warp` to every merging rank whose slice touches the head
     const int h = warp;
     const int o_lo = first_owner + (h * D) / per_o, o_hi = first_owner + (h * D + D - 1) / per_o;
     const int o = o_lo + lane;
     if (o <= o_hi) {
       float* dst = cluster.map_shared_rank(rml + (rank * G + h) * 2, o);
-      dst[0] = m_run;
-      dst[1] = l_run;
+      dst[0] = rM[h];
+      dst[1] = rL[h];
     }
   }
-  __syncthreads();
   for (int i = tid; i < E; i += kThreads) {
-    float sum = 0.f;
-    for (int k = 0; k < PVt::kSub; ++k) sum += red[k * E + i];
+    const int h = i / D;
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) a = fmaf(wf[w * G + h], wacc[w * E + i], a);
     const int ow = i / per_o;
-    *cluster.map_shared_rank(racc + rank * per_o + (i - ow * per_o), first_owner + ow) = sum;
+    *cluster.map_shared_rank(racc + rank * per_o + (i - ow * per_o), first_owner + ow) = a;
   }
   cluster.sync();  // #3: every partial pushed to this rank is visible
 
