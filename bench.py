@@ -434,6 +434,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
                "steps": n_e2e, "path": "compkv_decode_step via the Python binding, eager launches"}
 
+    # incremental append of one token per sequence (timed on a copy of one cache's summaries)
+    c0 = caches[0]
+    sa = ck.Summaries(*(t.clone() for t in (c0["summ"].mean_k, c0["summ"].var_g,
+                                            c0["summ"].mean_v, c0["summ"].count)))
+    k_new = c0["K"][:, :, -1].contiguous()
+    v_new = c0["V"][:, :, -1].contiguous()
+    pos = torch.full((wl.batch,), wl.ctx_len - 1, dtype=torch.int32, device=dev)
+    n_app = 200
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            ck.append(shape, k_new, v_new, pos, sa, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_app):
+            ck.append(shape, k_new, v_new, pos, sa, stream=stream)
+        e1.record(stream)
+    stream.synchronize()
+    append_us = e0.elapsed_time(e1) / n_app * 1e3
+    del sa
+
     status = max(ck.read_device_status(c["ws"], stream) for c in caches)
     if rank != 0:
         return
@@ -473,6 +493,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                   "frac_of_" + peak_src: nbytes["dense"] / (ms_dense / 1e3) / 1e9 / peak,
                   "speedup_sparse_over_dense": ms_dense / (ms / args.steps)},
         "build_summaries_ms": statistics.median(build_times),
+        "append_us": append_us,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
         "clocks": clocks, "device_status": status,
     }

@@ -78,6 +78,7 @@ typedef enum compkv_status {
 
 /* Device status bits recorded in the workspace status word by a kernel. */
 #define COMPKV_DEVERR_WAIT_TIMEOUT 0x1 /* an mbarrier wait gave up after its iteration limit   */
+#define COMPKV_DEVERR_BAD_POSITION 0x2 /* compkv_append: a position outside [0, T); skipped     */
 
 /* ------------------------------------------------------------------------------------------ */
 /* Sizes                                                                                       */
@@ -115,6 +116,28 @@ size_t compkv_full_workspace_bytes(const compkv_shape* shape);
 int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const void* K,
                            const void* V, const int32_t* ctx_lens, float* mean_k, float* var_g,
                            float* mean_v, int32_t* count, void* stream);
+
+/* a0, incremental. One new token per sequence enters the cache: its key and value update the
+ * summaries of the block that receives it (CompKV review, Frequently asked questions: the
+ * per-block summaries are "updated incrementally as new tokens enter the cache"). For each
+ * sequence b and kv-head g, with t = positions[b] and j = t / 16 (n = count[j] before the call):
+ *   n' = n + 1;  mu' = mu + (k - mu) / n';  nu' = nu + (v - nu) / n';
+ *   var_g[j, q]' = (n |C_q| var_g[j, q] + sum_{c in C_q} (k_c - mu_c)(k_c - mu'_c)) / (n' |C_q|)
+ * (Welford's update of the per-channel sums of squared deviations, summed over each group; exact
+ * from the stored (n, mu, var_g) because of the population-variance reading of var_g). A block
+ * with n = 0 becomes the token itself with zero variance. The caller appends tokens in order:
+ * t must be the sequence's current length, and every block before j must be full.
+ *   k_new, v_new  device [B, Hkv, d] of `dtype`: the new token's key and value
+ *   positions     device int32 [B]: t per sequence (the length before this token)
+ *   K, V          device [B, Hkv, T, d] caches of capacity T = shape->ctx_len, or NULL; when
+ *                 given, the token is also stored at row t
+ *   mean_k, var_g, mean_v, count   summaries as for compkv_build_summaries, updated in place
+ *   status        device int32 or NULL: a sequence with t outside [0, T) is skipped and
+ *                 COMPKV_DEVERR_BAD_POSITION is OR-ed into *status
+ * One warp per (sequence, kv-head); no workspace.                                              */
+int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_new,
+                  const void* v_new, const int32_t* positions, void* K, void* V, float* mean_k,
+                  float* var_g, float* mean_v, int32_t* count, int32_t* status, void* stream);
 
 /* a1 + a2. Compensation-aware score and Top-K selection, per (sequence, kv-head).
  * CompKV review, Summary (Section 3, Eq. 4-7: the residual of an omitted block is governed by its

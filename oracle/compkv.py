@@ -113,6 +113,42 @@ def block_summaries(k, v, block_size: int = 16, n_groups: int = 4) -> Summaries:
     return Summaries(count, mean_k, var_g, mean_v)
 
 
+def empty_summaries(nb: int, d: int, n_groups: int = 4) -> Summaries:
+    """Summaries of nb blocks that hold no token yet (n = 0, all moments 0)."""
+    return Summaries(np.zeros(nb, dtype=np.int64), np.zeros((nb, d)), np.zeros((nb, n_groups)),
+                     np.zeros((nb, d)))
+
+
+def append_token(summ: Summaries, t: int, k_t, v_t, block_size: int = 16) -> Summaries:
+    """The summaries of tokens [0, t] from those of [0, t) and token t (CompKV review, Frequently
+    asked questions: the per-block summaries are "updated incrementally as new tokens enter the
+    cache"). Returns a new Summaries; `summ` must have room for block t // block_size.
+
+    Welford's update of the running mean and of the sum of squared deviations per channel,
+        n' = n + 1,  mu' = mu + (k - mu) / n',  M2_c' = M2_c + (k_c - mu_c)(k_c - mu'_c),
+    aggregated over each channel group. The grouped variance (R4: the mean over the group of the
+    per-channel population variances) stays exactly updatable from (n, mu, var_g) alone, because
+    the group's sum of M2_c is n |C| var_g. The mean value is a plain running mean.
+    """
+    k_t, v_t = _f64(k_t), _f64(v_t)
+    j = t // block_size
+    count, mean_k = summ.count.copy(), summ.mean_k.copy()
+    var_g, mean_v = summ.var_g.copy(), summ.mean_v.copy()
+    r = var_g.shape[1]
+    d = mean_k.shape[1]
+    gs = d // r
+    n = int(count[j])
+    n1 = n + 1
+    mu = mean_k[j]
+    mu1 = mu + (k_t - mu) / n1
+    m2 = var_g[j] * (n * gs) + ((k_t - mu) * (k_t - mu1)).reshape(r, gs).sum(axis=1)
+    var_g[j] = m2 / (n1 * gs)
+    mean_k[j] = mu1
+    mean_v[j] = mean_v[j] + (v_t - mean_v[j]) / n1
+    count[j] = n1
+    return Summaries(count, mean_k, var_g, mean_v)
+
+
 # ----------------------------------------------------------------------------- scores
 
 def default_scale(d: int) -> float:

@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "compkv_workspace_bytes": (SZ, [SP, I32]),
             "compkv_full_workspace_bytes": (SZ, [SP]),
             "compkv_build_summaries": (ctypes.c_int, [SP, ctypes.c_int, P, P, P, P, P, P, P, P]),
+            "compkv_append": (ctypes.c_int, [SP, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P]),
             "compkv_score_select": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
                                                    I32, F, P, P, P, SZ, P]),
             "compkv_score_stream": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P, P, P,
@@ -191,6 +192,18 @@ def build_summaries(shape: LayerShape, K: torch.Tensor, V: torch.Tensor, out: Su
                                      _p(out.mean_k), _p(out.var_g), _p(out.mean_v), _p(out.count),
                                      _stream(stream)), "build_summaries")
     return out
+
+
+def append(shape: LayerShape, k_new: torch.Tensor, v_new: torch.Tensor, positions: torch.Tensor,
+           summ: Summaries, K: torch.Tensor | None = None, V: torch.Tensor | None = None,
+           status: torch.Tensor | None = None, stream=None) -> Summaries:
+    """One new token per sequence enters the cache: updates `summ` in place (and stores the token
+    at row positions[b] of K/V when given). positions: int32 [B] on the device."""
+    _ok(lib().compkv_append(ctypes.byref(shape.c()), _dt(k_new), _p(k_new), _p(v_new),
+                            _p(positions), _p(K), _p(V), _p(summ.mean_k), _p(summ.var_g),
+                            _p(summ.mean_v), _p(summ.count), _p(status), _stream(stream)),
+        "append")
+    return summ
 
 
 def score_select(shape: LayerShape, q: torch.Tensor, summ: Summaries, budget_tokens: int,

@@ -146,6 +146,39 @@ int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const 
   return cuda_status(compkv::launch_build_summaries(a, static_cast<cudaStream_t>(stream)));
 }
 
+int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_new,
+                  const void* v_new, const int32_t* positions, void* K, void* V, float* mean_k,
+                  float* var_g, float* mean_v, int32_t* count, int32_t* status, void* stream) {
+  int st = check_shape(shape);
+  if (st) return st;
+  if ((st = check_dtype(dtype))) return st;
+  if (!k_new || !v_new || !positions || !mean_k || !var_g || !mean_v || !count || (!K) != (!V))
+    return COMPKV_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned4(positions) || (K && !aligned16(K)) ||
+      (V && !aligned16(V)) || !aligned16(mean_k) || !aligned16(mean_v) || !aligned4(var_g) ||
+      !aligned4(count) || (status && !aligned4(status)))
+    return COMPKV_ERR_BAD_ALIGNMENT;
+  compkv::AppendArgs a;
+  a.bf16 = dtype == COMPKV_BF16;
+  a.pairs = shape->batch * shape->n_kv_heads;
+  a.Hkv = shape->n_kv_heads;
+  a.T = shape->ctx_len;
+  a.D = shape->head_dim;
+  a.Nb = n_blocks(shape);
+  a.r = shape->n_groups;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.positions = positions;
+  a.K = K;
+  a.V = V;
+  a.mean_k = mean_k;
+  a.var_g = var_g;
+  a.mean_v = mean_v;
+  a.count = count;
+  a.status = status;
+  return cuda_status(compkv::launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
 enum class Upto { kStream, kSelect, kAttend };
 
 // Streaming score kernel, then (unless `upto` is kStream) the select kernel, or with kAttend the

@@ -29,6 +29,21 @@ struct SummariesArgs {
   int32_t* count;
 };
 
+struct AppendArgs {
+  bool bf16;
+  int pairs, Hkv, T, D, Nb, r;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* positions;
+  void* K;
+  void* V;
+  float* mean_k;
+  float* var_g;
+  float* mean_v;
+  int32_t* count;
+  int32_t* status;
+};
+
 // A Mean-compensation partial per query head: [m, l, acc[D]] with m a reference logit,
 // l = sum n e^{lbar - m} and acc = sum n e^{lbar - m} nu over the blocks it covers.
 inline size_t comp_partial_floats(int G, int D) { return static_cast<size_t>(G) * (D + 2); }
@@ -130,6 +145,7 @@ int full_splits(int B, int Hkv, int T);
 inline int max_full_splits(int T) { return (T + 511) / 512; }
 
 cudaError_t launch_build_summaries(const SummariesArgs& a, cudaStream_t st);
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st);
 cudaError_t launch_decode_fused(const FusedArgs& a, cudaStream_t st);
 cudaError_t launch_full_decode(const FullArgs& a, cudaStream_t st);

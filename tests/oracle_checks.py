@@ -7,6 +7,7 @@ What pins what (sources: CompKV abstract and the Evolve.pub review of CompKV):
 
 * summaries      -> numpy mean/var per block (library), identical keys give exact zeros,
                     partial last block counts, hand-derived closed forms (golden files).
+* append         -> token-by-token Welford appends equal the rebuilt summaries (review, FAQ).
 * scores         -> golden closed forms; second-order behaviour: score x Zhat / R_j -> 1 as the
                     within-block spread eps -> 0 with error O(eps) (O(eps^2) for symmetric
                     spreads), and the mass estimate's error shrinks as eps^3 (eps^4).
@@ -84,6 +85,31 @@ def check_summaries_identical_keys():
     # variance is zero up to (ulps * |k|)^2
     bound = (16 * np.finfo(np.float64).eps * np.max(np.abs(k))) ** 2
     assert np.all(s.var_g <= bound), s.var_g
+
+
+def check_append_equals_rebuild():
+    """Appending tokens one at a time (Welford) gives the block summaries of the longer sequence,
+    from an empty cache and from a partly filled one (review, FAQ: summaries updated
+    incrementally as new tokens enter the cache). Pinned to block_summaries (itself pinned to
+    numpy), for several group counts and a partial last block."""
+    rng = np.random.default_rng(41)
+    for d, r, T0, T1 in ((8, 4, 0, 37), (16, 2, 21, 70), (16, 16, 16, 33), (12, 3, 5, 6)):
+        _, k, v = _rand_cache(rng, T1, d, offset=2.0)
+        k = k * 3.0 + 5.0  # a large common offset: a naive sum-of-squares update loses digits
+        nb = -(-T1 // 16)
+        s = O.empty_summaries(nb, d, r)
+        if T0:
+            base = O.block_summaries(k[:T0], v[:T0], 16, r)
+            nb0 = base.count.shape[0]
+            s.count[:nb0], s.mean_k[:nb0] = base.count, base.mean_k
+            s.var_g[:nb0], s.mean_v[:nb0] = base.var_g, base.mean_v
+        for t in range(T0, T1):
+            s = O.append_token(s, t, k[t], v[t], 16)
+        ref = O.block_summaries(k, v, 16, r)
+        assert np.array_equal(s.count, ref.count), (s.count, ref.count)
+        _close(s.mean_k, ref.mean_k, rtol=1e-12, atol=1e-12, what="append mean_k")
+        _close(s.mean_v, ref.mean_v, rtol=1e-12, atol=1e-12, what="append mean_v")
+        _close(s.var_g, ref.var_g, rtol=1e-10, atol=1e-12, what="append var_g")
 
 
 def check_golden_two_blocks():
@@ -337,7 +363,8 @@ def check_gqa_normalisation():
     assert set(O.select_blocks(raw, kb)) != set(best)
 
 
-ALL_CHECKS = [check_summaries_library, check_summaries_identical_keys, check_golden_two_blocks,
+ALL_CHECKS = [check_summaries_library, check_summaries_identical_keys, check_append_equals_rebuild,
+              check_golden_two_blocks,
               check_golden_grouped_variance, check_kl_identity,
               check_second_form_and_dense_limit, check_zero_residual_block, check_ties_and_order,
               check_second_order_limit, check_bruteforce_residual_topk,

@@ -15,7 +15,7 @@ import oracle_checks as C
 _orig = {name: getattr(O, name) for name in (
     "block_summaries", "logit_variance_estimate", "second_order_log_mass", "head_scores",
     "compensated_attention", "select_blocks", "block_mean_logits", "dense_attention",
-    "group_scores", "token_logits", "block_residuals", "log_partitions")}
+    "group_scores", "token_logits", "block_residuals", "log_partitions", "append_token")}
 
 
 def _summaries_sample_var(k, v, block_size=16, n_groups=4):
@@ -108,7 +108,37 @@ def _logits_no_scale(q, k, scale):
     return _orig["token_logits"](q, k, 1.0)
 
 
+def _append_squared_new_mean(summ, t, k_t, v_t, block_size=16):
+    """Welford slip: (k - mu')^2 instead of (k - mu)(k - mu')."""
+    s = _orig["append_token"](summ, t, k_t, v_t, block_size)
+    j = t // block_size
+    n1 = s.count[j]
+    if n1 > 1:
+        k_t = np.asarray(k_t, dtype=float)
+        r = s.var_g.shape[1]
+        gs = s.mean_k.shape[1] // r
+        mu = summ.mean_k[j]
+        mu1 = s.mean_k[j]
+        wrong = ((k_t - mu1) ** 2).reshape(r, gs).sum(1)
+        right = ((k_t - mu) * (k_t - mu1)).reshape(r, gs).sum(1)
+        s.var_g[j] = s.var_g[j] + (wrong - right) / (n1 * gs)
+    return s
+
+
+def _append_mean_over_n(summ, t, k_t, v_t, block_size=16):
+    """Running-mean slip: divides by the old count."""
+    s = _orig["append_token"](summ, t, k_t, v_t, block_size)
+    j = t // block_size
+    n = summ.count[j]
+    if n > 0:
+        v_t = np.asarray(v_t, dtype=float)
+        s.mean_v[j] = summ.mean_v[j] + (v_t - summ.mean_v[j]) / n
+    return s
+
+
 MUTATIONS = {
+    "append_squared_new_mean": ("append_token", _append_squared_new_mean),
+    "append_mean_over_old_count": ("append_token", _append_mean_over_n),
     "sample_variance": ("block_summaries", _summaries_sample_var),
     "interleaved_groups": ("block_summaries", _summaries_interleaved),
     "vhat_missing_scale": ("logit_variance_estimate", _vhat_one_scale),
