@@ -13,4 +13,5 @@ from .compkv import (MODES, Summaries, StepResult, block_summaries, block_mean_l
                      dense_attention, compensated_distribution, kl_divergence, log_partitions,
                      block_residuals, brute_force_best_subset, decode_step, dense_step,
                      default_scale, n_blocks, block_bounds, logsumexp, empty_summaries,
-                     append_token)
+                     append_token, average_ranks, rank_correlation, residual_capture,
+                     group_residual_criterion)

@@ -315,6 +315,51 @@ def block_residuals(q, k, scale: float, block_size: int = 16) -> tuple[np.ndarra
     return mass, resid
 
 
+# ----------------------------------------------------------------------------- diagnostics
+
+def average_ranks(x) -> np.ndarray:
+    """Ranks 1..n of x ascending; tied values share the mean of their ranks."""
+    x = np.asarray(x, dtype=np.float64)
+    order = np.argsort(x, kind="stable")
+    ranks = np.empty(x.shape[0])
+    i = 0
+    while i < x.shape[0]:
+        j = i
+        while j + 1 < x.shape[0] and x[order[j + 1]] == x[order[i]]:
+            j += 1
+        ranks[order[i:j + 1]] = (i + j) / 2.0 + 1.0
+        i = j + 1
+    return ranks
+
+
+def rank_correlation(a, b) -> float:
+    """Spearman's rank correlation: Pearson's correlation of the average ranks (the fidelity
+    statistic the review quotes for App. B.2, 0.8604 on real activations)."""
+    ra, rb = average_ranks(a), average_ranks(b)
+    ra, rb = ra - ra.mean(), rb - rb.mean()
+    den = math.sqrt(float((ra * ra).sum()) * float((rb * rb).sum()))
+    return float((ra * rb).sum() / den) if den > 0 else 0.0
+
+
+def residual_capture(score, resid, k_sel: int) -> float:
+    """Share of the best achievable omitted-residual reduction that Top-K by `score` achieves:
+    sum of resid over Top-K(score) / sum of resid over Top-K(resid) (review, App. B.2: 81.53%
+    residual capture at r = 4 on real activations)."""
+    resid = np.asarray(resid, dtype=np.float64)
+    best = resid[select_blocks(resid, k_sel)].sum()
+    got = resid[select_blocks(score, k_sel)].sum()
+    return float(got / best) if best > 0 else 1.0
+
+
+def group_residual_criterion(q_group, k, scale: float, block_size: int = 16) -> np.ndarray:
+    """T_j = sum over the group's heads of R_{j,h} / Z_h: the first-order change of sum_h KL_h
+    when block j is omitted under Mean compensation (readings 1 and 6). What the group score S_j
+    estimates."""
+    q_group = np.atleast_2d(_f64(q_group))
+    k = _f64(k)
+    return sum(block_residuals(q_group[h], k, scale, block_size)[1] for h in range(q_group.shape[0]))
+
+
 def brute_force_best_subset(q_heads, k, k_sel: int, scale: float, block_size: int = 16,
                             compensate: bool = True) -> tuple[tuple, float]:
     """Enumerate every K_b-subset of blocks; return the one minimising sum_h KL(q_S^h || p^h).

@@ -363,9 +363,31 @@ def check_gqa_normalisation():
     assert set(O.select_blocks(raw, kb)) != set(best)
 
 
+def check_fidelity_statistics():
+    """Spearman and residual capture: closed forms and textbook cases (App. B.2 statistics)."""
+    x = np.array([3.0, 1.0, 4.0, 1.5, 9.0, 2.6])
+    assert abs(O.rank_correlation(x, x) - 1.0) < 1e-15
+    assert abs(O.rank_correlation(x, -x) + 1.0) < 1e-15
+    assert abs(O.rank_correlation(x, np.exp(x)) - 1.0) < 1e-15          # monotone invariance
+    # n = 4, one swapped pair: 1 - 6 sum d^2 / (n (n^2 - 1)) = 1 - 6*2/60 = 0.8
+    assert abs(O.rank_correlation([1, 2, 3, 4], [1, 3, 2, 4]) - 0.8) < 1e-15
+    # ties share the mean rank: ranks of [5, 7, 7, 9] are [1, 2.5, 2.5, 4]
+    assert np.array_equal(O.average_ranks([5, 7, 7, 9]), [1, 2.5, 2.5, 4])
+    # pearson of ranks [1, 2.5, 2.5, 4] vs [1, 2, 3, 4]: 4.5 / sqrt(4.5 * 5)
+    assert abs(O.rank_correlation([5, 7, 7, 9], [1, 2, 3, 4]) - 4.5 / math.sqrt(22.5)) < 1e-15
+    R = np.array([0.5, 0.1, 0.3, 0.05, 0.2])
+    assert O.residual_capture(R, R, 2) == 1.0
+    assert abs(O.residual_capture(-R, R, 2) - (0.1 + 0.05) / (0.5 + 0.3)) < 1e-15
+    assert abs(O.residual_capture([0, 0, 0, 1, 1], R, 2) - (0.05 + 0.2) / 0.8) < 1e-15
+    # the group criterion of one head is that head's normalised residual
+    rng = np.random.default_rng(5)
+    q, k, _ = _rand_cache(rng, 64, 8)
+    _close(O.group_residual_criterion(q, k, 0.3), O.block_residuals(q, k, 0.3)[1], what="T_j")
+
+
 ALL_CHECKS = [check_summaries_library, check_summaries_identical_keys, check_append_equals_rebuild,
               check_golden_two_blocks,
               check_golden_grouped_variance, check_kl_identity,
               check_second_form_and_dense_limit, check_zero_residual_block, check_ties_and_order,
               check_second_order_limit, check_bruteforce_residual_topk,
-              check_mass_only_reduction, check_gqa_normalisation]
+              check_mass_only_reduction, check_gqa_normalisation, check_fidelity_statistics]

@@ -15,7 +15,8 @@ import oracle_checks as C
 _orig = {name: getattr(O, name) for name in (
     "block_summaries", "logit_variance_estimate", "second_order_log_mass", "head_scores",
     "compensated_attention", "select_blocks", "block_mean_logits", "dense_attention",
-    "group_scores", "token_logits", "block_residuals", "log_partitions", "append_token")}
+    "group_scores", "token_logits", "block_residuals", "log_partitions", "append_token", "rank_correlation",
+    "residual_capture")}
 
 
 def _summaries_sample_var(k, v, block_size=16, n_groups=4):
@@ -136,7 +137,21 @@ def _append_mean_over_n(summ, t, k_t, v_t, block_size=16):
     return s
 
 
+def _spearman_on_values(a, b):
+    """Pearson on raw values instead of ranks."""
+    a, b = np.asarray(a, dtype=float), np.asarray(b, dtype=float)
+    a, b = a - a.mean(), b - b.mean()
+    return float((a * b).sum() / np.sqrt((a * a).sum() * (b * b).sum()))
+
+
+def _capture_unnormalised(score, resid, k_sel):
+    resid = np.asarray(resid, dtype=float)
+    return float(resid[O.select_blocks(score, k_sel)].sum())
+
+
 MUTATIONS = {
+    "spearman_on_values": ("rank_correlation", _spearman_on_values),
+    "capture_unnormalised": ("residual_capture", _capture_unnormalised),
     "append_squared_new_mean": ("append_token", _append_squared_new_mean),
     "append_mean_over_old_count": ("append_token", _append_mean_over_n),
     "sample_variance": ("block_summaries", _summaries_sample_var),
