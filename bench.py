@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense-steps", type=int, default=200)
+    ap.add_argument("--summary-dtype", default="fp32", choices=["fp32", "fp16"],
+                    help="storage of the mean key / mean value summaries")
     return ap.parse_args()
 
 
@@ -62,15 +64,17 @@ def workload(name: str, budget):
     return wl if budget is None else wl.with_(budget=budget, name=f"{wl.name}_b{budget}")
 
 
-def step_bytes(wl) -> dict:
-    """Algorithmic bytes of one step: fp32 summaries of every block, bf16 K/V of the selected
-    blocks, q in, out (fp32) out. Intermediates (workspace partials) are not counted."""
+def step_bytes(wl, summary_dtype: str = "fp32") -> dict:
+    """Algorithmic bytes of one step: every block's summaries (mean key and mean value in the
+    summary dtype, fp32 grouped variances, int32 count), bf16 K/V of the selected blocks, q in,
+    out (fp32) out. Intermediates (workspace partials) are not counted."""
     esz = 2 if wl.dtype == "bf16" else 4
+    ssz = 2 if summary_dtype == "fp16" else 4
     nb = wl.n_blocks
     kb = min(wl.budget // 16, nb)
     pairs = wl.batch * wl.n_kv_heads
     d, r = wl.head_dim, wl.n_groups
-    summ = pairs * nb * 4 * (2 * d + r + 1)
+    summ = pairs * nb * (ssz * 2 * d + 4 * (r + 1))
     sel_kv = pairs * kb * 16 * d * esz * 2
     q = wl.batch * wl.n_q_heads * d * esz
     out = wl.batch * wl.n_q_heads * d * 4
@@ -241,11 +245,11 @@ def cpu_oracle_sample(wl, target_s: float, max_units: int | None = None) -> dict
                       f"{wl.name}, summaries prebuilt, numpy fp64, BLAS limited to 1 thread"}
 
 
-def config_of(wl) -> dict:
+def config_of(wl, summary_dtype: str = "fp32") -> dict:
     return {"workload": wl.name, "batch": wl.batch, "n_q_heads": wl.n_q_heads,
             "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "ctx_len": wl.ctx_len,
             "budget_tokens": wl.budget, "block_size": wl.block_size, "n_groups": wl.n_groups,
-            "input_dtype": wl.dtype, "summary_dtype": "fp32",
+            "input_dtype": wl.dtype, "summary_dtype": summary_dtype,
             "l2": f"rotates {N_CACHES} independent caches; working set "
                   f"{N_CACHES} x step bytes > 126 MB L2",
             "graph": "CUDA graphs; streaming score kernel, then the select-and-attend kernel with programmatic dependent launch"}
@@ -269,7 +273,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = workload(args.workload, args.budget)
-    shape = ck.LayerShape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ctx_len, wl.n_groups)
+    shape = ck.LayerShape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.ctx_len, wl.n_groups,
+                          summary_dtype=args.summary_dtype)
     kb = ck.num_selected(shape, wl.budget)
     stream = torch.cuda.Stream(device=dev)
 
@@ -458,7 +463,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank != 0:
         return
 
-    nbytes = step_bytes(wl)
+    nbytes = step_bytes(wl, args.summary_dtype)
     peaks = measured_peaks()
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
@@ -477,7 +482,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "metric": METRIC, "value": throughput(world, args.steps, ms), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": config_of(wl),
+        "data": "synthetic", "config": config_of(wl, args.summary_dtype),
         "hbm": {"gbs": gbs_step, "bytes_per_step": nbytes["step"], "peak_gbs": peak,
                 "frac_of_" + peak_src: gbs_step / peak, "frac_of_nominal_8000": gbs_step / 8000.0},
         "roofline": {"kernel": "score_stream_kernel (scores, records and compensation partials "

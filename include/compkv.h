@@ -48,7 +48,13 @@ typedef struct compkv_shape {
                       /* given                                                                 */
   int32_t block_size; /* must be 16                                                            */
   int32_t n_groups;   /* r: a power of two with 1 <= r <= d (default 4)                        */
+  int32_t summary_dtype; /* compkv_summary_dtype of mean_k and mean_v (0 = fp32)                */
 } compkv_shape;
+
+/* Storage type of the mean key and mean value summaries (the grouped variances stay fp32, the
+ * counts int32). FP16 halves the bytes the score pass streams; values are rounded to nearest
+ * even when stored and computed on in fp32. */
+typedef enum compkv_summary_dtype { COMPKV_SUMMARY_FP32 = 0, COMPKV_SUMMARY_FP16 = 1 } compkv_summary_dtype;
 
 /* Element type of q, K and V (summaries and outputs are always fp32). */
 typedef enum compkv_dtype { COMPKV_BF16 = 0, COMPKV_FP32 = 1 } compkv_dtype;
@@ -111,11 +117,12 @@ size_t compkv_full_workspace_bytes(const compkv_shape* shape);
  * Blocks with n_j = 0 get zeros.
  *   K, V      device, [B, Hkv, T, d] of `dtype`, read once
  *   ctx_lens  device int32 [B] (T_b, 1..T) or NULL for T_b = T
- *   mean_k, mean_v  device fp32 [B, Hkv, N_b, d];  var_g device fp32 [B, Hkv, N_b, r];
+ *   mean_k, mean_v  device [B, Hkv, N_b, d] of shape->summary_dtype (fp32 or fp16);
+ *                   var_g device fp32 [B, Hkv, N_b, r];
  *   count     device int32 [B, Hkv, N_b]                                                       */
 int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const void* K,
-                           const void* V, const int32_t* ctx_lens, float* mean_k, float* var_g,
-                           float* mean_v, int32_t* count, void* stream);
+                           const void* V, const int32_t* ctx_lens, void* mean_k, float* var_g,
+                           void* mean_v, int32_t* count, void* stream);
 
 /* a0, incremental. One new token per sequence enters the cache: its key and value update the
  * summaries of the block that receives it (CompKV review, Frequently asked questions: the
@@ -136,8 +143,8 @@ int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const 
  *                 COMPKV_DEVERR_BAD_POSITION is OR-ed into *status
  * One warp per (sequence, kv-head); no workspace.                                              */
 int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_new,
-                  const void* v_new, const int32_t* positions, void* K, void* V, float* mean_k,
-                  float* var_g, float* mean_v, int32_t* count, int32_t* status, void* stream);
+                  const void* v_new, const int32_t* positions, void* K, void* V, void* mean_k,
+                  float* var_g, void* mean_v, int32_t* count, int32_t* status, void* stream);
 
 /* a1 + a2. Compensation-aware score and Top-K selection, per (sequence, kv-head).
  * CompKV review, Summary (Section 3, Eq. 4-7: the residual of an omitted block is governed by its
@@ -160,8 +167,8 @@ int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_n
  *   scores     device fp32 [B, Hkv, N_b] receives S_j, or NULL
  *   workspace  device, >= compkv_workspace_bytes(shape, budget_tokens)                         */
 int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                        const void* q, const float* mean_k, const float* var_g,
-                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        const void* q, const void* mean_k, const float* var_g,
+                        const void* mean_v, const int32_t* count, int32_t budget_tokens,
                         float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
                         size_t workspace_bytes, void* stream);
 
@@ -172,8 +179,8 @@ int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
  * step) can be timed on its own; a following compkv_score_select recomputes everything it needs.
  * Arguments as for compkv_score_select.                                                       */
 int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                        const void* q, const float* mean_k, const float* var_g,
-                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        const void* q, const void* mean_k, const float* var_g,
+                        const void* mean_v, const int32_t* count, int32_t budget_tokens,
                         float softmax_scale, void* workspace, size_t workspace_bytes,
                         void* stream);
 
@@ -191,8 +198,8 @@ int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
  *   mean_k, mean_v, count  summaries (only the selected blocks' rows are read here)
  *   out       device fp32 [B, Hq, d]                                                          */
 int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                         const void* q, const void* K, const void* V, const float* mean_k,
-                         const float* mean_v, const int32_t* count, const int32_t* sel_idx,
+                         const void* q, const void* K, const void* V, const void* mean_k,
+                         const void* mean_v, const int32_t* count, const int32_t* sel_idx,
                          int32_t budget_tokens, float softmax_scale, float* out, void* workspace,
                          size_t workspace_bytes, void* stream);
 
@@ -201,8 +208,8 @@ int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_m
  * programmatic dependent launch so its prologue overlaps the first's tail; the selection is kept
  * on chip and also written to sel_idx). Arguments as above. */
 int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                       const void* q, const void* K, const void* V, const float* mean_k,
-                       const float* var_g, const float* mean_v, const int32_t* count,
+                       const void* q, const void* K, const void* V, const void* mean_k,
+                       const float* var_g, const void* mean_v, const int32_t* count,
                        int32_t budget_tokens, float softmax_scale, int32_t* sel_idx,
                        float* scores, float* out, void* workspace, size_t workspace_bytes,
                        void* stream);
@@ -240,8 +247,8 @@ int compkv_full_decode(const compkv_shape* shape, compkv_dtype dtype, const void
  *     threads) race on the array: the caller must serialise them.
  * Arguments and outputs are those of compkv_decode_step without workspace and workspace_bytes. */
 int compkv_decode_step_static(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                              const void* q, const void* K, const void* V, const float* mean_k,
-                              const float* var_g, const float* mean_v, const int32_t* count,
+                              const void* q, const void* K, const void* V, const void* mean_k,
+                              const float* var_g, const void* mean_v, const int32_t* count,
                               int32_t budget_tokens, float softmax_scale, int32_t* sel_idx,
                               float* scores, float* out, void* stream);
 

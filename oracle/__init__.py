@@ -14,4 +14,4 @@ from .compkv import (MODES, Summaries, StepResult, block_summaries, block_mean_l
                      block_residuals, brute_force_best_subset, decode_step, dense_step,
                      default_scale, n_blocks, block_bounds, logsumexp, empty_summaries,
                      append_token, average_ranks, rank_correlation, residual_capture,
-                     group_residual_criterion)
+                     group_residual_criterion, store)

@@ -87,10 +87,22 @@ class Summaries:
     mean_v: np.ndarray   # [Nb, d] nu_j, mean value
 
 
-def block_summaries(k, v, block_size: int = 16, n_groups: int = 4) -> Summaries:
+def store(x: np.ndarray, storage: str) -> np.ndarray:
+    """Storage rounding of a mean key / mean value: "fp32" keeps fp64 (the fp32 kernel's own
+    rounding is inside the tolerances), "fp16" rounds to the nearest fp16 (IEEE, ties to even)."""
+    if storage == "fp32":
+        return x
+    if storage == "fp16":
+        return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+    raise ValueError(storage)
+
+
+def block_summaries(k, v, block_size: int = 16, n_groups: int = 4,
+                    storage: str = "fp32") -> Summaries:
     """Mean key, grouped key variance and mean value of every block [Summary; FAQ].
 
-    k, v: [T, d] for one sequence and kv-head. Population (1/n) variances (R4).
+    k, v: [T, d] for one sequence and kv-head. Population (1/n) variances (R4), computed from
+    the exact mean; `storage` rounds the stored means (the variance stays exact).
     """
     k, v = _f64(k), _f64(v)
     T, d = k.shape
@@ -108,8 +120,8 @@ def block_summaries(k, v, block_size: int = 16, n_groups: int = 4) -> Summaries:
         mu = kb.mean(axis=0)
         chan_var = ((kb - mu) ** 2).mean(axis=0)
         var_g[j] = chan_var.reshape(n_groups, d // n_groups).mean(axis=1)
-        mean_k[j] = mu
-        mean_v[j] = vb.mean(axis=0)
+        mean_k[j] = store(mu, storage)
+        mean_v[j] = store(vb.mean(axis=0), storage)
     return Summaries(count, mean_k, var_g, mean_v)
 
 
@@ -119,7 +131,8 @@ def empty_summaries(nb: int, d: int, n_groups: int = 4) -> Summaries:
                      np.zeros((nb, d)))
 
 
-def append_token(summ: Summaries, t: int, k_t, v_t, block_size: int = 16) -> Summaries:
+def append_token(summ: Summaries, t: int, k_t, v_t, block_size: int = 16,
+                 storage: str = "fp32") -> Summaries:
     """The summaries of tokens [0, t] from those of [0, t) and token t (CompKV review, Frequently
     asked questions: the per-block summaries are "updated incrementally as new tokens enter the
     cache"). Returns a new Summaries; `summ` must have room for block t // block_size.
@@ -143,8 +156,8 @@ def append_token(summ: Summaries, t: int, k_t, v_t, block_size: int = 16) -> Sum
     mu1 = mu + (k_t - mu) / n1
     m2 = var_g[j] * (n * gs) + ((k_t - mu) * (k_t - mu1)).reshape(r, gs).sum(axis=1)
     var_g[j] = m2 / (n1 * gs)
-    mean_k[j] = mu1
-    mean_v[j] = mean_v[j] + (v_t - mean_v[j]) / n1
+    mean_k[j] = store(mu1, storage)
+    mean_v[j] = store(mean_v[j] + (v_t - mean_v[j]) / n1, storage)
     count[j] = n1
     return Summaries(count, mean_k, var_g, mean_v)
 
@@ -396,7 +409,7 @@ class StepResult:
 
 def decode_step(q, K, V, budget: int, block_size: int = 16, n_groups: int = 4,
                 scale: float | None = None, mode: str = "compkv", ctx_lens=None,
-                selection=None, pairs=None, summaries=None) -> StepResult:
+                selection=None, pairs=None, summaries=None, storage: str = "fp32") -> StepResult:
     """One CompKV decode step for a batch, summaries -> score -> Top-K -> compensated attention.
 
     q [B, Hq, d]; K, V [B, Hkv, T, d]. ``ctx_lens`` gives each sequence's token count (default
@@ -420,7 +433,7 @@ def decode_step(q, K, V, budget: int, block_size: int = 16, n_groups: int = 4,
         vb = _f64(V[b, g, :Tb])
         qg = _f64(q[b, g * G:(g + 1) * G])
         summ = (summaries[b][g] if summaries is not None
-                else block_summaries(kb, vb, block_size, n_groups))
+                else block_summaries(kb, vb, block_size, n_groups, storage))
         S = group_scores(qg, summ, s, mode)
         chosen = (np.asarray(selection[b][g]) if selection is not None
                   else select_blocks(S, n_select(budget, block_size, summ.count.shape[0])))

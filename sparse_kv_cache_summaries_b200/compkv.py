@@ -19,6 +19,7 @@ LIB_PATH = pathlib.Path(__file__).resolve().with_name("libcompkv.so")
 HEADER = pathlib.Path(__file__).resolve().parent.parent / "include" / "compkv.h"
 
 MODES = {"compkv": 0, "mass": 1, "mass_comp": 2}
+SUMMARY_DTYPES = {"fp32": 0, "fp16": 1}
 _DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 BLOCK_SIZE = 16
 
@@ -36,7 +37,7 @@ class Shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("ctx_len", ctypes.c_int32), ("block_size", ctypes.c_int32),
-                ("n_groups", ctypes.c_int32)]
+                ("n_groups", ctypes.c_int32), ("summary_dtype", ctypes.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -49,6 +50,7 @@ class LayerShape:
     ctx_len: int
     n_groups: int = 4
     block_size: int = BLOCK_SIZE
+    summary_dtype: str = "fp32"  # storage of mean_k / mean_v: "fp32" or "fp16"
 
     @property
     def n_blocks(self) -> int:
@@ -60,7 +62,7 @@ class LayerShape:
 
     def c(self) -> Shape:
         return Shape(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.ctx_len,
-                     self.block_size, self.n_groups)
+                     self.block_size, self.n_groups, SUMMARY_DTYPES[self.summary_dtype])
 
 
 _lib = None
@@ -161,17 +163,18 @@ def full_workspace_bytes(shape: LayerShape) -> int:
 
 @dataclasses.dataclass
 class Summaries:
-    mean_k: torch.Tensor   # [B, Hkv, Nb, d] fp32
+    mean_k: torch.Tensor   # [B, Hkv, Nb, d] fp32 or fp16 (LayerShape.summary_dtype)
     var_g: torch.Tensor    # [B, Hkv, Nb, r] fp32
-    mean_v: torch.Tensor   # [B, Hkv, Nb, d] fp32
+    mean_v: torch.Tensor   # [B, Hkv, Nb, d] fp32 or fp16
     count: torch.Tensor    # [B, Hkv, Nb] int32
 
 
 def empty_summaries(shape: LayerShape, device="cuda") -> Summaries:
     B, H, nb, d, r = shape.batch, shape.n_kv_heads, shape.n_blocks, shape.head_dim, shape.n_groups
     f = dict(device=device, dtype=torch.float32)
-    return Summaries(torch.empty((B, H, nb, d), **f), torch.empty((B, H, nb, r), **f),
-                     torch.empty((B, H, nb, d), **f),
+    m = dict(device=device, dtype=torch.float16 if shape.summary_dtype == "fp16" else torch.float32)
+    return Summaries(torch.empty((B, H, nb, d), **m), torch.empty((B, H, nb, r), **f),
+                     torch.empty((B, H, nb, d), **m),
                      torch.empty((B, H, nb), device=device, dtype=torch.int32))
 
 

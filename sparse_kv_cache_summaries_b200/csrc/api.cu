@@ -34,6 +34,8 @@ int check_shape(const compkv_shape* s) {
   if (s->block_size != compkv::kBlockTokensHost) return COMPKV_ERR_UNSUPPORTED_SHAPE;
   const int r = s->n_groups;
   if ((r & (r - 1)) != 0 || r > s->head_dim) return COMPKV_ERR_UNSUPPORTED_SHAPE;
+  if (s->summary_dtype != COMPKV_SUMMARY_FP32 && s->summary_dtype != COMPKV_SUMMARY_FP16)
+    return COMPKV_ERR_INVALID_ARG;
   // grid and index limits of the kernels
   const long long nb = (s->ctx_len + 15) / 16;
   if (static_cast<long long>(s->batch) * s->n_kv_heads * nb > (1LL << 30)) return COMPKV_ERR_UNSUPPORTED_SHAPE;
@@ -119,8 +121,8 @@ size_t compkv_full_workspace_bytes(const compkv_shape* shape) {
 }
 
 int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const void* K,
-                           const void* V, const int32_t* ctx_lens, float* mean_k, float* var_g,
-                           float* mean_v, int32_t* count, void* stream) {
+                           const void* V, const int32_t* ctx_lens, void* mean_k, float* var_g,
+                           void* mean_v, int32_t* count, void* stream) {
   int st = check_shape(shape);
   if (st) return st;
   if ((st = check_dtype(dtype))) return st;
@@ -130,6 +132,7 @@ int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const 
     return COMPKV_ERR_BAD_ALIGNMENT;
   compkv::SummariesArgs a;
   a.bf16 = dtype == COMPKV_BF16;
+  a.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
   a.B = shape->batch;
   a.Hkv = shape->n_kv_heads;
   a.T = shape->ctx_len;
@@ -147,8 +150,8 @@ int compkv_build_summaries(const compkv_shape* shape, compkv_dtype dtype, const 
 }
 
 int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_new,
-                  const void* v_new, const int32_t* positions, void* K, void* V, float* mean_k,
-                  float* var_g, float* mean_v, int32_t* count, int32_t* status, void* stream) {
+                  const void* v_new, const int32_t* positions, void* K, void* V, void* mean_k,
+                  float* var_g, void* mean_v, int32_t* count, int32_t* status, void* stream) {
   int st = check_shape(shape);
   if (st) return st;
   if ((st = check_dtype(dtype))) return st;
@@ -160,6 +163,7 @@ int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_n
     return COMPKV_ERR_BAD_ALIGNMENT;
   compkv::AppendArgs a;
   a.bf16 = dtype == COMPKV_BF16;
+  a.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
   a.pairs = shape->batch * shape->n_kv_heads;
   a.Hkv = shape->n_kv_heads;
   a.T = shape->ctx_len;
@@ -184,8 +188,8 @@ enum class Upto { kStream, kSelect, kAttend };
 // Streaming score kernel, then (unless `upto` is kStream) the select kernel, or with kAttend the
 // select-and-attend kernel, launched with programmatic dependent launch.
 static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                             const void* q, const float* mean_k, const float* var_g,
-                             const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                             const void* q, const void* mean_k, const float* var_g,
+                             const void* mean_v, const int32_t* count, int32_t budget_tokens,
                              float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
                              size_t workspace_bytes, void* stream, Upto upto, const void* K,
                              const void* V, float* out) {
@@ -204,6 +208,7 @@ static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, comp
   int nctas = 0;
   compkv::StreamArgs a;
   a.bf16 = dtype == COMPKV_BF16;
+  a.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
   a.mode = mode;
   a.pairs = pairs;
   a.G = c.G;
@@ -228,6 +233,7 @@ static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, comp
   if (rc || upto == Upto::kStream) return rc;
   compkv::FusedArgs b;
   b.bf16 = a.bf16;
+  b.fp16_summ = a.fp16_summ;
   b.mode = mode;
   b.do_select = true;
   b.do_attend = upto == Upto::kAttend;
@@ -258,8 +264,8 @@ static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, comp
 }
 
 int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                        const void* q, const float* mean_k, const float* var_g,
-                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        const void* q, const void* mean_k, const float* var_g,
+                        const void* mean_v, const int32_t* count, int32_t budget_tokens,
                         float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
                         size_t workspace_bytes, void* stream) {
   return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
@@ -268,8 +274,8 @@ int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
 }
 
 int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                        const void* q, const float* mean_k, const float* var_g,
-                        const float* mean_v, const int32_t* count, int32_t budget_tokens,
+                        const void* q, const void* mean_k, const float* var_g,
+                        const void* mean_v, const int32_t* count, int32_t budget_tokens,
                         float softmax_scale, void* workspace, size_t workspace_bytes,
                         void* stream) {
   return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
@@ -278,8 +284,8 @@ int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
 }
 
 int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                         const void* q, const void* K, const void* V, const float* mean_k,
-                         const float* mean_v, const int32_t* count, const int32_t* sel_idx,
+                         const void* q, const void* K, const void* V, const void* mean_k,
+                         const void* mean_v, const int32_t* count, const int32_t* sel_idx,
                          int32_t budget_tokens, float softmax_scale, float* out, void* workspace,
                          size_t workspace_bytes, void* stream) {
   Common c;
@@ -294,6 +300,7 @@ int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_m
   const compkv::StepWorkspace W = step_ws(shape);
   compkv::FusedArgs b;
   b.bf16 = dtype == COMPKV_BF16;
+  b.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
   b.mode = mode;
   b.do_select = false;
   b.do_attend = true;
@@ -324,8 +331,8 @@ int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_m
 }
 
 int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                       const void* q, const void* K, const void* V, const float* mean_k,
-                       const float* var_g, const float* mean_v, const int32_t* count,
+                       const void* q, const void* K, const void* V, const void* mean_k,
+                       const float* var_g, const void* mean_v, const int32_t* count,
                        int32_t budget_tokens, float softmax_scale, int32_t* sel_idx,
                        float* scores, float* out, void* workspace, size_t workspace_bytes,
                        void* stream) {

@@ -11,7 +11,7 @@
 namespace compkv {
 namespace {
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendArgs p) {
   constexpr int VW = D / 32;
   __shared__ float dev_s[kWarps][D];  // per-channel (k - mu)(k - mu') of each warp's pair
@@ -44,15 +44,16 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
   const size_t row = static_cast<size_t>(pair) * p.Nb + j;
   const int n = p.count[row];
   const float n1 = static_cast<float>(n + 1);
-  float* mk = p.mean_k + row * D + lane * VW;
-  float* mv = p.mean_v + row * D + lane * VW;
+  S* mk = static_cast<S*>(p.mean_k) + row * D + lane * VW;
+  S* mv = static_cast<S*>(p.mean_v) + row * D + lane * VW;
 #pragma unroll
   for (int e = 0; e < VW; ++e) {
-    const float mu = mk[e];
+    const float mu = sload(mk + e);  // the stored mean (fp16 storage: already rounded)
     const float mu1 = mu + (k[e] - mu) / n1;
     dev_s[warp][lane * VW + e] = (k[e] - mu) * (k[e] - mu1);
-    mk[e] = mu1;
-    mv[e] = mv[e] + (v[e] - mv[e]) / n1;
+    sstore(mk + e, mu1);
+    const float nu = sload(mv + e);
+    sstore(mv + e, nu + (v[e] - nu) / n1);
   }
   __syncwarp();
   const int gs = D / p.r;
@@ -66,11 +67,11 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
   if (lane == 0) p.count[row] = n + 1;
 }
 
-template <typename T>
+template <typename T, typename S>
 cudaError_t launch_t(const AppendArgs& a, cudaStream_t st) {
   const dim3 grid((a.pairs + kWarps - 1) / kWarps);
-  if (a.D == 128) append_kernel<T, 128><<<grid, kThreads, 0, st>>>(a);
-  else append_kernel<T, 64><<<grid, kThreads, 0, st>>>(a);
+  if (a.D == 128) append_kernel<T, 128, S><<<grid, kThreads, 0, st>>>(a);
+  else append_kernel<T, 64, S><<<grid, kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -78,7 +79,8 @@ cudaError_t launch_t(const AppendArgs& a, cudaStream_t st) {
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st) {
   if (a.D != 64 && a.D != 128) return cudaErrorInvalidValue;
-  return a.bf16 ? launch_t<uint16_t>(a, st) : launch_t<float>(a, st);
+  if (a.fp16_summ) return a.bf16 ? launch_t<uint16_t, __half>(a, st) : launch_t<float, __half>(a, st);
+  return a.bf16 ? launch_t<uint16_t, float>(a, st) : launch_t<float, float>(a, st);
 }
 
 }  // namespace compkv

@@ -3,6 +3,7 @@
 // bf16 unpacking, warp/CTA reductions and an order-preserving float key.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -192,6 +193,12 @@ __device__ __forceinline__ void unpack8_bf16(const uint4& w, float (&f)[8]) {
     f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
   }
 }
+
+// Summary storage of the mean key and mean value: fp32, or fp16 rounded to nearest even.
+__device__ __forceinline__ float sload(const float* p) { return *p; }
+__device__ __forceinline__ float sload(const __half* p) { return __half2float(*p); }
+__device__ __forceinline__ void sstore(float* p, float x) { *p = x; }
+__device__ __forceinline__ void sstore(__half* p, float x) { *p = __float2half_rn(x); }
 
 __device__ __forceinline__ float to_float(float x) { return x; }
 __device__ __forceinline__ float to_float(uint16_t x) {

@@ -107,7 +107,7 @@ struct FParams {
   const void* q;
   const void* K;
   const void* V;
-  const float* mean_v;
+  const void* mean_v;  // [pairs][Nb][D] of the summary type
   const float* u;
   const float* xrec;
   const float* zpart;
@@ -159,7 +159,7 @@ __device__ __forceinline__ int stream_cta_of_tile(long long f, int nctas, int F)
 }
 
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, typename S>  // S: summary storage type (float or __half)
 __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_constant__ FParams p) {
   constexpr int XS = xrec_stride(G);
   extern __shared__ __align__(128) unsigned char sm[];
@@ -515,7 +515,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   using RP = RowPart<T, VEP>;
   const T* Kbase = static_cast<const T*>(p.K) + static_cast<size_t>(pr) * p.T * D;
   const T* Vbase = static_cast<const T*>(p.V) + static_cast<size_t>(pr) * p.T * D;
-  const float* NUbase = p.mean_v + static_cast<size_t>(pr) * p.Nb * D;
+  const S* NUbase = static_cast<const S*>(p.mean_v) + static_cast<size_t>(pr) * p.Nb * D;
   const float* XRbase = p.xrec + static_cast<size_t>(pr) * p.Nb * XS;
   float qv[G][VEP];
 #pragma unroll
@@ -556,9 +556,9 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     for (int e = 0; e < VEP; ++e) nu[e] = 0.f;
     if (compensate && first && j >= 0) {
       xh = __ldg(rec + my_h);
-      const float* nrow = NUbase + static_cast<size_t>(j) * D + lane * VEP;
+      const S* nrow = NUbase + static_cast<size_t>(j) * D + lane * VEP;
 #pragma unroll
-      for (int e = 0; e < VEP; ++e) nu[e] = __ldg(nrow + e);
+      for (int e = 0; e < VEP; ++e) nu[e] = sload(nrow + e);
     }
     // logits: partial dots over this lane's channels, one transpose-reduce for the group
     float v[NV];
@@ -727,22 +727,27 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 const void* kptr_g(int G) {
   switch (G) {
-    case 1: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 1>);
-    case 2: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 2>);
-    case 4: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 4>);
-    case 8: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 8>);
+    case 1: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 1, S>);
+    case 2: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 2, S>);
+    case 4: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 4, S>);
+    case 8: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 8, S>);
   }
   return nullptr;
 }
 
 int ksub_of(bool bf16, int D) { return kThreads / (D / (bf16 ? 2 : 1)); }
 
-const void* pick(bool bf16, int D, int G) {
-  if (bf16) return D == 128 ? kptr_g<uint16_t, 128>(G) : (D == 64 ? kptr_g<uint16_t, 64>(G) : nullptr);
-  return D == 128 ? kptr_g<float, 128>(G) : (D == 64 ? kptr_g<float, 64>(G) : nullptr);
+template <typename S>
+const void* pick_s(bool bf16, int D, int G) {
+  if (bf16) return D == 128 ? kptr_g<uint16_t, 128, S>(G) : (D == 64 ? kptr_g<uint16_t, 64, S>(G) : nullptr);
+  return D == 128 ? kptr_g<float, 128, S>(G) : (D == 64 ? kptr_g<float, 64, S>(G) : nullptr);
+}
+
+const void* pick(bool bf16, int D, int G, bool fp16) {
+  return fp16 ? pick_s<__half>(bf16, D, G) : pick_s<float>(bf16, D, G);
 }
 
 // Launch plan of one problem shape: the cluster size and the shared-memory layout.
@@ -813,7 +818,7 @@ cudaError_t make_plan(const void* kern, const FusedArgs& a, Plan* out) {
 }  // namespace
 
 cudaError_t launch_decode_fused(const FusedArgs& a, cudaStream_t st) {
-  const void* kern = pick(a.bf16, a.D, a.G);
+  const void* kern = pick(a.bf16, a.D, a.G, a.fp16_summ);
   if (!kern) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);

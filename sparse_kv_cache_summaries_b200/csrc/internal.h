@@ -19,27 +19,29 @@ __host__ __device__ constexpr int xrec_stride(int G) { return ((G + 1 + 3) / 4) 
 
 struct SummariesArgs {
   bool bf16;
+  bool fp16_summ;  // mean_k / mean_v stored as fp16
   int B, Hkv, T, D, Nb, r;
   const void* K;
   const void* V;
   const int32_t* ctx_lens;
-  float* mean_k;
+  void* mean_k;
   float* var_g;
-  float* mean_v;
+  void* mean_v;
   int32_t* count;
 };
 
 struct AppendArgs {
   bool bf16;
+  bool fp16_summ;  // mean_k / mean_v stored as fp16
   int pairs, Hkv, T, D, Nb, r;
   const void* k_new;
   const void* v_new;
   const int32_t* positions;
   void* K;
   void* V;
-  float* mean_k;
+  void* mean_k;
   float* var_g;
-  float* mean_v;
+  void* mean_v;
   int32_t* count;
   int32_t* status;
 };
@@ -50,13 +52,14 @@ inline size_t comp_partial_floats(int G, int D) { return static_cast<size_t>(G) 
 
 struct StreamArgs {
   bool bf16;
+  bool fp16_summ;  // mean_k / mean_v stored as fp16
   int mode;
   int pairs, G, D, Nb, r, slots;
   float scale;
   const void* q;
-  const float* mean_k;
+  const void* mean_k;
   const float* var_g;
-  const float* mean_v;
+  const void* mean_v;
   const int32_t* count;
   float* u;          // [pairs][Nb][G]   per-block log scores
   float* xrec;       // [pairs][Nb][xrec_stride(G)]
@@ -72,6 +75,7 @@ struct StreamArgs {
 // sel_idx and `comp` as given).
 struct FusedArgs {
   bool bf16;
+  bool fp16_summ;  // mean_k / mean_v stored as fp16
   int mode;
   bool do_select, do_attend;
   int pairs, G, D, T, Nb, Kb, slots, nctas_stream;
@@ -79,7 +83,7 @@ struct FusedArgs {
   const void* q;
   const void* K;
   const void* V;
-  const float* mean_v;
+  const void* mean_v;
   const float* u;
   const float* xrec;      // [pairs][Nb][xrec_stride(G)] from the streaming kernel
   const float* zpart;
@@ -139,7 +143,7 @@ struct StepWorkspace {
 };
 
 // Grid size of the streaming score kernel for this shape on the current device.
-int stream_grid_ctas(bool bf16, int D, int G, int r, int total_tiles);
+int stream_grid_ctas(bool bf16, bool fp16_summ, int D, int G, int r, int total_tiles);
 // Splits per kv-head of full_decode (<= max_full_splits(T)).
 int full_splits(int B, int Hkv, int T);
 inline int max_full_splits(int T) { return (T + 511) / 512; }

@@ -38,8 +38,8 @@ int scratch_for_current_device(void** out) {
 
 extern "C" int compkv_decode_step_static(const compkv_shape* shape, compkv_dtype dtype,
                                          compkv_mode mode, const void* q, const void* K,
-                                         const void* V, const float* mean_k, const float* var_g,
-                                         const float* mean_v, const int32_t* count,
+                                         const void* V, const void* mean_k, const float* var_g,
+                                         const void* mean_v, const int32_t* count,
                                          int32_t budget_tokens, float softmax_scale,
                                          int32_t* sel_idx, float* scores, float* out,
                                          void* stream) {

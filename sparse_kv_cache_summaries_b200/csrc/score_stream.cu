@@ -46,9 +46,9 @@ struct StreamParams {
   int mode, Nb, tiles_per_pair, total_tiles, nctas, slots, r;
   float scale;
   const void* q;
-  const float* mean_k;
+  const void* mean_k;   // [pairs][Nb][D] of the summary type
   const float* var_g;
-  const float* mean_v;
+  const void* mean_v;
   const int32_t* count;
   float* u;        // [pairs][Nb][G]
   float* xrec;     // [pairs][Nb][xrec_stride(G)]  {x_0..x_{G-1}, n}
@@ -61,12 +61,15 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast
 
 struct SLay {
   size_t stage_bytes, off_mu, off_nu, off_var, off_cnt, stage0, full, rel, wsw, q, qn, refw, red, logn, total;
-  __host__ __device__ void build(int D, int G, int r) {
+  __host__ __device__ void build(int D, int G, int r, int ssz) {
     off_mu = 0;
-    off_nu = a16(sizeof(float) * kTile * D);
-    off_var = a16(off_nu + sizeof(float) * kTile * D);
+    off_nu = a16(static_cast<size_t>(ssz) * kTile * D);
+    off_var = a16(off_nu + static_cast<size_t>(ssz) * kTile * D);
     off_cnt = a16(off_var + sizeof(float) * kTile * r);
     stage_bytes = a16(off_cnt + sizeof(int) * kTile);
+    // a released stage is the segment merge's scratch: [kWarps][G][D] floats
+    const size_t scratch = sizeof(float) * kWarps * G * D;
+    if (stage_bytes < scratch) stage_bytes = a16(scratch);
     size_t o = 0;
     full = o;   o = a16(o + 8 * kStages);
     rel = o;    o = a16(o + sizeof(uint32_t) * (kStages + 2));  // release counters, abort, issued
@@ -82,11 +85,34 @@ struct SLay {
 };
 
 // R = 4 specialises the default group count (grouped variances as one float4); R = 0 is any r.
-template <typename TQ, int D, int G, int R>
+// One lane's VW channels of a summary row in shared memory, as VW / 2 float pairs.
+template <int VW, typename S>
+__device__ __forceinline__ void row_pairs(const S* row, float2 (&a)[VW / 2]) {
+  if constexpr (sizeof(S) == 4) {
+    if constexpr (VW == 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(row);
+      a[0] = make_float2(a4.x, a4.y);
+      a[1] = make_float2(a4.z, a4.w);
+    } else {
+      a[0] = *reinterpret_cast<const float2*>(row);
+    }
+  } else {
+    if constexpr (VW == 4) {
+      const uint2 w = *reinterpret_cast<const uint2*>(row);
+      a[0] = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+      a[1] = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+    } else {
+      a[0] = __half22float2(*reinterpret_cast<const __half2*>(row));
+    }
+  }
+}
+
+// S: storage type of the mean key and mean value (float, or __half).
+template <typename TQ, int D, int G, int R, typename S>
 __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_constant__ StreamParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   SLay L;
-  L.build(D, G, p.r);
+  L.build(D, G, p.r, sizeof(S));
   const int r = p.r;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool compensate = p.mode != COMPKV_MODE_MASS;
@@ -121,10 +147,11 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     for (int i = lane; i < tn * r; i += 32) cp_async4(var_d + i, p.var_g + row0 * r + i);
     for (int i = lane; i < tn; i += 32) cp_async4(cnt_d + i, p.count + row0 + i);
     if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(tn) * D * sizeof(float);
+      const uint32_t bytes = static_cast<uint32_t>(tn) * D * sizeof(S);
       mbar_arrive_expect_tx(&full[st], compensate ? 2 * bytes : bytes);
-      bulk_g2s_stream(sb + L.off_mu, p.mean_k + row0 * D, bytes, &full[st], policy);
-      if (compensate) bulk_g2s_stream(sb + L.off_nu, p.mean_v + row0 * D, bytes, &full[st], policy);
+      bulk_g2s_stream(sb + L.off_mu, static_cast<const S*>(p.mean_k) + row0 * D, bytes, &full[st], policy);
+      if (compensate)
+        bulk_g2s_stream(sb + L.off_nu, static_cast<const S*>(p.mean_v) + row0 * D, bytes, &full[st], policy);
     }
     cp_async_arrive(&full[st]);
   };
@@ -302,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     const int jt0 = (f % TP) * kTile;
     const int tn = ok ? min(kTile, p.Nb - jt0) : 0;
     const unsigned char* sb = sm + L.stage0 + L.stage_bytes * st;
-    const float* mu_t = reinterpret_cast<const float*>(sb + L.off_mu);
-    const float* nu_t = reinterpret_cast<const float*>(sb + L.off_nu);
+    const S* mu_t = reinterpret_cast<const S*>(sb + L.off_mu);
+    const S* nu_t = reinterpret_cast<const S*>(sb + L.off_nu);
     const float* var_t = reinterpret_cast<const float*>(sb + L.off_var);
     const int* cnt_t = reinterpret_cast<const int*>(sb + L.off_cnt);
     const int jw = warp * kBlocksPerWarp;  // the warp's first block in the tile
@@ -312,15 +339,8 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     float v[NVAL];
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b) {
-      const float* row = mu_t + (jw + b) * D + lane * VW;
       float2 a[VW / 2];
-      if constexpr (VW == 4) {
-        const float4 a4 = reinterpret_cast<const float4*>(row)[0];
-        a[0] = make_float2(a4.x, a4.y);
-        a[1] = make_float2(a4.z, a4.w);
-      } else {
-        a[0] = reinterpret_cast<const float2*>(row)[0];
-      }
+      row_pairs<VW, S>(mu_t + (jw + b) * D + lane * VW, a);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         float2 s2 = __fmul2_rn(qv[hh][0], a[0]);
@@ -397,15 +417,8 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
 #pragma unroll
       for (int b = 0; b < kBlocksPerWarp; ++b) {
         if (jw + b < tn) {
-          const float* row = nu_t + (jw + b) * D + lane * VW;
           float2 a[VW / 2];
-          if constexpr (VW == 4) {
-            const float4 a4 = reinterpret_cast<const float4*>(row)[0];
-            a[0] = make_float2(a4.x, a4.y);
-            a[1] = make_float2(a4.z, a4.w);
-          } else {
-            a[0] = reinterpret_cast<const float2*>(row)[0];
-          }
+          row_pairs<VW, S>(nu_t + (jw + b) * D + lane * VW, a);
           float wb[G];
           if constexpr (G % 4 == 0) {
 #pragma unroll
@@ -465,19 +478,20 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   if (cur >= 0) finish_segment(0);
 }
 
-template <typename TQ, int D, int G>
+template <typename TQ, int D, int G, typename S>
 const void* kptr(int r) {
-  return r == 4 ? reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G, 4>)
-                : reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G, 0>);
+  return r == 4 ? reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G, 4, S>)
+                : reinterpret_cast<const void*>(&score_stream_kernel<TQ, D, G, 0, S>);
 }
 
-const void* pick(bool bf16, int D, int G, int r) {
+template <typename S>
+const void* pick_s(bool bf16, int D, int G, int r) {
 #define COMPKV_PICK(T, DD)                  \
   switch (G) {                              \
-    case 1: return kptr<T, DD, 1>(r);       \
-    case 2: return kptr<T, DD, 2>(r);       \
-    case 4: return kptr<T, DD, 4>(r);       \
-    case 8: return kptr<T, DD, 8>(r);       \
+    case 1: return kptr<T, DD, 1, S>(r);    \
+    case 2: return kptr<T, DD, 2, S>(r);    \
+    case 4: return kptr<T, DD, 4, S>(r);    \
+    case 8: return kptr<T, DD, 8, S>(r);    \
   }
   if (bf16) {
     if (D == 128) { COMPKV_PICK(uint16_t, 128) } else { COMPKV_PICK(uint16_t, 64) }
@@ -486,6 +500,10 @@ const void* pick(bool bf16, int D, int G, int r) {
   }
 #undef COMPKV_PICK
   return nullptr;
+}
+
+const void* pick(bool bf16, int D, int G, int r, bool fp16) {
+  return fp16 ? pick_s<__half>(bf16, D, G, r) : pick_s<float>(bf16, D, G, r);
 }
 
 struct Grid {
@@ -498,7 +516,7 @@ Grid g_grids[16];
 int g_ngrids = 0;
 std::mutex g_mu;
 
-cudaError_t grid_for(const void* kern, int D, int G, int r, Grid* out) {
+cudaError_t grid_for(const void* kern, int D, int G, int r, bool fp16, Grid* out) {
   int dev = 0;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lock(g_mu);
@@ -512,7 +530,7 @@ cudaError_t grid_for(const void* kern, int D, int G, int r, Grid* out) {
   g.dev = dev;
   g.r = r;
   SLay L;
-  L.build(D, G, r);
+  L.build(D, G, r, fp16 ? 2 : 4);
   g.smem = L.total;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(g.smem));
   if (e != cudaSuccess) return e;
@@ -535,10 +553,10 @@ int stream_ctas(int total_tiles, int sms, int ctas_per_sm) {
 }  // namespace
 
 cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
-  const void* kern = pick(a.bf16, a.D, a.G, a.r);
+  const void* kern = pick(a.bf16, a.D, a.G, a.r, a.fp16_summ);
   if (!kern) return cudaErrorInvalidValue;
   Grid g;
-  cudaError_t e = grid_for(kern, a.D, a.G, a.r, &g);
+  cudaError_t e = grid_for(kern, a.D, a.G, a.r, a.fp16_summ, &g);
   if (e != cudaSuccess) return e;
   StreamParams p;
   p.mode = a.mode;
@@ -570,10 +588,10 @@ cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
-int stream_grid_ctas(bool bf16, int D, int G, int r, int total_tiles) {
-  const void* kern = pick(bf16, D, G, r);
+int stream_grid_ctas(bool bf16, bool fp16_summ, int D, int G, int r, int total_tiles) {
+  const void* kern = pick(bf16, D, G, r, fp16_summ);
   Grid g;
-  if (!kern || grid_for(kern, D, G, r, &g) != cudaSuccess) return -1;
+  if (!kern || grid_for(kern, D, G, r, fp16_summ, &g) != cudaSuccess) return -1;
   return stream_ctas(total_tiles, g.sms, g.ctas_per_sm);
 }
 

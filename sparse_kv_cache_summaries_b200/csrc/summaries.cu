@@ -38,12 +38,12 @@ __device__ __forceinline__ void to_floats<float, 4>(const uint4& w, float (&f)[4
   f[3] = __uint_as_float(w.w);
 }
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 __global__ void __launch_bounds__(kThreads)
     build_summaries_kernel(const T* __restrict__ K, const T* __restrict__ V,
                            const int32_t* __restrict__ ctx_lens, int n_blk_total, int Hkv, int T_cap,
-                           int Nb, int r, float* __restrict__ mean_k, float* __restrict__ var_g,
-                           float* __restrict__ mean_v, int32_t* __restrict__ count) {
+                           int Nb, int r, S* __restrict__ mean_k, float* __restrict__ var_g,
+                           S* __restrict__ mean_v, int32_t* __restrict__ count) {
   using Gm = Geom<T, D>;
   constexpr int EPV = Gm::kEpv, LPR = Gm::kLpr, RPL = Gm::kRpl, NL = Gm::kLoads;
   const int lane = threadIdx.x & 31;
@@ -125,12 +125,22 @@ __global__ void __launch_bounds__(kThreads)
 
   const size_t row_out = static_cast<size_t>(w);
   if (rs == 0) {
-    float4* mk = reinterpret_cast<float4*>(mean_k + row_out * D + li * EPV);
-    float4* mv = reinterpret_cast<float4*>(mean_v + row_out * D + li * EPV);
+    if constexpr (sizeof(S) == 4) {
+      float4* mk = reinterpret_cast<float4*>(mean_k + row_out * D + li * EPV);
+      float4* mv = reinterpret_cast<float4*>(mean_v + row_out * D + li * EPV);
 #pragma unroll
-    for (int e = 0; e < EPV; e += 4) {
-      mk[e / 4] = make_float4(mu[e], mu[e + 1], mu[e + 2], mu[e + 3]);
-      mv[e / 4] = make_float4(vs[e] * inv_n, vs[e + 1] * inv_n, vs[e + 2] * inv_n, vs[e + 3] * inv_n);
+      for (int e = 0; e < EPV; e += 4) {
+        mk[e / 4] = make_float4(mu[e], mu[e + 1], mu[e + 2], mu[e + 3]);
+        mv[e / 4] = make_float4(vs[e] * inv_n, vs[e + 1] * inv_n, vs[e + 2] * inv_n, vs[e + 3] * inv_n);
+      }
+    } else {  // fp16 storage: pairs rounded to nearest even
+      __half2* mk = reinterpret_cast<__half2*>(mean_k + row_out * D + li * EPV);
+      __half2* mv = reinterpret_cast<__half2*>(mean_v + row_out * D + li * EPV);
+#pragma unroll
+      for (int e = 0; e < EPV; e += 2) {
+        mk[e / 2] = __floats2half2_rn(mu[e], mu[e + 1]);
+        mv[e / 2] = __floats2half2_rn(vs[e] * inv_n, vs[e + 1] * inv_n);
+      }
     }
   }
   if (lane == 0) count[row_out] = n;
@@ -155,23 +165,26 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 cudaError_t launch_t(const SummariesArgs& a, cudaStream_t st) {
   const int total = a.B * a.Hkv * a.Nb;
   const int grid = (total + kWarps - 1) / kWarps;
-  build_summaries_kernel<T, D><<<grid, kThreads, 0, st>>>(
+  build_summaries_kernel<T, D, S><<<grid, kThreads, 0, st>>>(
       static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.ctx_lens, total, a.Hkv, a.T, a.Nb,
-      a.r, a.mean_k, a.var_g, a.mean_v, a.count);
+      a.r, static_cast<S*>(a.mean_k), a.var_g, static_cast<S*>(a.mean_v), a.count);
   return cudaGetLastError();
+}
+
+template <typename S>
+cudaError_t launch_s(const SummariesArgs& a, cudaStream_t st) {
+  if (a.bf16) return a.D == 128 ? launch_t<uint16_t, 128, S>(a, st) : launch_t<uint16_t, 64, S>(a, st);
+  return a.D == 128 ? launch_t<float, 128, S>(a, st) : launch_t<float, 64, S>(a, st);
 }
 
 }  // namespace
 
 cudaError_t launch_build_summaries(const SummariesArgs& a, cudaStream_t st) {
-  if (a.bf16) {
-    return a.D == 128 ? launch_t<uint16_t, 128>(a, st) : launch_t<uint16_t, 64>(a, st);
-  }
-  return a.D == 128 ? launch_t<float, 128>(a, st) : launch_t<float, 64>(a, st);
+  return a.fp16_summ ? launch_s<__half>(a, st) : launch_s<float>(a, st);
 }
 
 }  // namespace compkv

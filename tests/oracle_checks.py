@@ -363,6 +363,23 @@ def check_gqa_normalisation():
     assert set(O.select_blocks(raw, kb)) != set(best)
 
 
+def check_fp16_storage():
+    """fp16 storage rounds the stored means exactly as numpy's IEEE fp16 cast does (ties to even),
+    leaves the variance (computed from the exact mean) and the counts untouched, and an append
+    over fp16 storage works from the stored, rounded means."""
+    rng = np.random.default_rng(8)
+    _, k, v = _rand_cache(rng, 40, 8)
+    a = O.block_summaries(k, v, 16, 2)
+    h = O.block_summaries(k, v, 16, 2, storage="fp16")
+    assert np.array_equal(h.mean_k, a.mean_k.astype(np.float16).astype(np.float64))
+    assert np.array_equal(h.mean_v, a.mean_v.astype(np.float16).astype(np.float64))
+    assert np.array_equal(h.var_g, a.var_g) and np.array_equal(h.count, a.count)
+    assert np.float16(1.0 + 2.0 ** -11) == np.float16(1.0)          # tie rounds to even
+    s = O.append_token(h, 40, k[0], v[0], 16, storage="fp16")
+    mu = h.mean_k[2] + (k[0] - h.mean_k[2]) / (h.count[2] + 1)
+    assert np.array_equal(s.mean_k[2], mu.astype(np.float16).astype(np.float64))
+
+
 def check_fidelity_statistics():
     """Spearman and residual capture: closed forms and textbook cases (App. B.2 statistics)."""
     x = np.array([3.0, 1.0, 4.0, 1.5, 9.0, 2.6])
@@ -390,4 +407,5 @@ ALL_CHECKS = [check_summaries_library, check_summaries_identical_keys, check_app
               check_golden_grouped_variance, check_kl_identity,
               check_second_form_and_dense_limit, check_zero_residual_block, check_ties_and_order,
               check_second_order_limit, check_bruteforce_residual_topk,
-              check_mass_only_reduction, check_gqa_normalisation, check_fidelity_statistics]
+              check_mass_only_reduction, check_gqa_normalisation, check_fidelity_statistics,
+              check_fp16_storage]

@@ -50,9 +50,9 @@ class GpuRun:
     ws: torch.Tensor | None = None
 
 
-def upload(wl: synth.Workload, ctx_lens=None, tensors=None) -> GpuRun:
+def upload(wl: synth.Workload, ctx_lens=None, tensors=None, summary_dtype="fp32") -> GpuRun:
     q, K, V = tensors if tensors is not None else synth.make_batch(wl)
-    shape = layer_shape(wl)
+    shape = layer_shape(wl, summary_dtype=summary_dtype)
     cl = None if ctx_lens is None else torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
     return GpuRun(wl, shape, q, K, V, q.cuda(), K.cuda(), V.cuda(), cl)
 
@@ -94,13 +94,14 @@ def check_summaries(run: GpuRun, pairs, tol=SUMM_TOL) -> dict:
     T = run.shape.ctx_len
     for b, g in pairs:
         Tb = T if run.ctx_lens is None else int(run.ctx_lens[b])
-        ref = oracle.block_summaries(run.K[b, g, :Tb], run.V[b, g, :Tb], 16, run.shape.n_groups)
+        ref = oracle.block_summaries(run.K[b, g, :Tb], run.V[b, g, :Tb], 16, run.shape.n_groups,
+                                     run.shape.summary_dtype)
         nb = ref.count.shape[0]
         cnt = run.summ.count[b, g].cpu().numpy()
         assert np.array_equal(cnt[:nb], ref.count), (b, g)
         assert np.all(cnt[nb:] == 0)
         for name in worst:
-            gpu = getattr(run.summ, name)[b, g, :nb].cpu().numpy()
+            gpu = getattr(run.summ, name)[b, g, :nb].float().cpu().numpy()
             e = rel_err(gpu, getattr(ref, name))
             worst[name] = max(worst[name], e)
             assert e <= tol, (name, b, g, e)
@@ -135,7 +136,8 @@ def check_step(run: GpuRun, budget: int, mode: str, pairs) -> dict:
     ref_scores = {}
     for b, g in pairs:
         Tb = s.ctx_len if run.ctx_lens is None else int(run.ctx_lens[b])
-        summ = oracle.block_summaries(run.K[b, g, :Tb], run.V[b, g, :Tb], 16, s.n_groups)
+        summ = oracle.block_summaries(run.K[b, g, :Tb], run.V[b, g, :Tb], 16, s.n_groups,
+                                      s.summary_dtype)
         S = oracle.group_scores(run.q[b, g * G:(g + 1) * G], summ, oracle.default_scale(s.head_dim),
                                 mode)
         ref_scores[(b, g)] = S
@@ -152,7 +154,7 @@ def check_step(run: GpuRun, budget: int, mode: str, pairs) -> dict:
         assert rel_err(sc_all[b, g, :nb], S) <= SCORE_RTOL, (b, g)
     ctx = None if run.ctx_lens is None else run.ctx_lens.cpu().numpy()
     res = oracle.decode_step(run.q, run.K, run.V, budget, 16, s.n_groups, mode=mode, ctx_lens=ctx,
-                             selection=selection, pairs=list(pairs))
+                             selection=selection, pairs=list(pairs), storage=s.summary_dtype)
     for b, g in pairs:
         ref = res.out[b, g * G:(g + 1) * G]
         got = out_all[b, g * G:(g + 1) * G]
