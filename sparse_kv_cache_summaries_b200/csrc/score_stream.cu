@@ -134,9 +134,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   const uint64_t policy = l2_evict_first_policy();
 
   // Refills the stage of local tile k (one whole warp).
-  auto issue = [&](int k) {
-    const int f = f0 + k;
-    const int pr = f / TP, t = f % TP;
+  auto issue = [&](int k, int pr, int t) {  // tile k is tile t of pair pr
     const int jt0 = t * kTile;
     const int tn = min(kTile, p.Nb - jt0);
     const size_t row0 = static_cast<size_t>(pr) * p.Nb + jt0;
@@ -167,8 +165,23 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   }
   if (tid < 17) logn_s[tid] = tid > 0 ? logf(static_cast<float>(tid)) : -CUDART_INF_F;
   __syncthreads();
+  // (pair, tile within the pair) of tile k + d, from those of tile k
+  auto advance = [&](int pr, int t, int d, int& pr_out, int& t_out) {
+    t += d;
+    while (t >= TP) {
+      t -= TP;
+      ++pr;
+    }
+    pr_out = pr;
+    t_out = t;
+  };
+  const int pr0 = f0 / TP, t0 = f0 % TP;
   if (warp == 0)
-    for (int k = 0; k < min(nt, kStages); ++k) issue(k);
+    for (int k = 0; k < min(nt, kStages); ++k) {
+      int pk, tk;
+      advance(pr0, t0, k, pk, tk);
+      issue(k, pk, tk);
+    }
   pdl_launch_dependents();
 
   // Lane map: lane l holds channels [l VW, l VW + VW) of every row for all G heads (a warp-wide
@@ -304,10 +317,10 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   // `ok` goes false (for this warp) once a wait gives up; the warp then stops waiting and
   // computing but keeps the loop's structure, so every CTA barrier stays matched.
   bool ok = true;
+  int pr = pr0, tt = t0;      // pair and tile-in-pair of tile k, kept without divisions
+  int st = 0, ph = 0;         // ring stage and its phase parity for tile k
 #pragma unroll 1
   for (int k = 0; k < nt; ++k) {
-    const int f = f0 + k;
-    const int pr = f / TP;
     if (pr != cur) {  // every warp reaches this at the same tile
       __syncthreads();
       // the stage of tile k - 1 is free: its refill waits until this segment switch is done
@@ -315,18 +328,19 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       start_segment(pr);
       cur = pr;
       if (warp == 0 && k >= 1 && k + kStages - 1 < nt && *abort_s == 0) {
-        issue(k + kStages - 1);
+        int pk, tk;
+        advance(pr, tt, kStages - 1, pk, tk);
+        issue(k + kStages - 1, pk, tk);
         if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(k + kStages));
       }
     }
-    const int st = k % kStages;
-    bool got = ok && mbar_wait(&full[st], (k / kStages) & 1, p.status);
+    bool got = ok && mbar_wait(&full[st], ph, p.status);
     got = __all_sync(0xffffffffu, got);
     if (!got && ok) {
       ok = false;
       if (lane == 0) *abort_s = 1;
     }
-    const int jt0 = (f % TP) * kTile;
+    const int jt0 = tt * kTile;
     const int tn = ok ? min(kTile, p.Nb - jt0) : 0;
     const unsigned char* sb = sm + L.stage0 + L.stage_bytes * st;
     const S* mu_t = reinterpret_cast<const S*>(sb + L.off_mu);
@@ -454,10 +468,12 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     before = __shfl_sync(0xffffffffu, before, 0);
     if (before % kWarps == kWarps - 1) {
       const int kk = k + kStages;
-      const bool defer = k + 1 < nt && (f + 1) / TP != pr;
+      const bool defer = k + 1 < nt && tt + 1 == TP;
       if (kk < nt && !defer && *abort_s == 0) {
         fence_proxy_async();
-        issue(kk);
+        int pk, tk;
+        advance(pr, tt, kStages, pk, tk);
+        issue(kk, pk, tk);
         if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(kk + 1));
       }
     }
@@ -466,6 +482,14 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       p.u[row * G + my_h] = st_u;
       p.xrec[row * XS + my_h] = xs;
       if (my_h == 0) p.xrec[row * XS + G] = __int_as_float(st_n);
+    }
+    if (++tt == TP) {
+      tt = 0;
+      ++pr;
+    }
+    if (++st == kStages) {
+      st = 0;
+      ph ^= 1;
     }
   }
   __syncthreads();
