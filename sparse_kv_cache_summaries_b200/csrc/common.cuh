@@ -561,11 +561,26 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Asynchronous store into another CTA's shared memory (shared::cluster addresses from
+// cluster_smem_addr), completing `bytes` of transactions on that CTA's mbarrier: the receiver
+// waits on its own mbarrier for the bytes it expects; no cluster barrier and no release fence.
+__device__ __forceinline__ void st_async_b32(uint32_t dst, uint32_t v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               ::"r"(dst), "r"(v), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void st_async_b64(uint32_t dst, uint64_t v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];"
+               ::"r"(dst), "l"(v), "r"(bar) : "memory");
+}
+
 // Split cluster barrier (all threads of every CTA of the cluster). An early relaxed arrive and a
 // later wait cost almost nothing; after the wait every CTA of the cluster has started, so its
 // shared memory may be written remotely.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
@@ -639,6 +654,35 @@ __device__ __forceinline__ int warp_sort_asc(int v) {
 // This CTA's 32 best codes of items [0, n) (code_at(i)), descending, in lists[0..31]. Each warp
 // scans a contiguous run in chunks of 32 (sort, merge into its running list); the 8 warp lists
 // then merge pairwise in 3 levels. `lists` needs kWarps * 32 entries. Contains CTA barriers.
+// Named CTA barriers over `n` threads (a multiple of 32): a producer arrives, a consumer waits.
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// The 8 warps' descending lists (`best` in each warp) merged pairwise in 3 levels; at level s
+// warp w (w % 2s == 0) takes warp w + s's list through `lists` and a named barrier (ids 1..7)
+// shared by those two warps only. Warp 0 returns the CTA's best 32; the other warps' return
+// values are partial. No CTA-wide barrier.
+__device__ __forceinline__ uint64_t warp_pairs_merge_top32(uint64_t best, uint64_t* lists) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int id = 1;
+#pragma unroll
+  for (int s = 1; s < kWarps; s <<= 1) {
+    if ((warp & (2 * s - 1)) == s) {  // producer at this level, done afterwards
+      lists[warp * 32 + lane] = best;
+      named_bar_arrive(id + (warp - s) / (2 * s), 64);
+    } else if ((warp & (2 * s - 1)) == 0) {
+      named_bar_sync(id + warp / (2 * s), 64);
+      best = warp_merge_top32(best, lists[(warp + s) * 32 + lane]);
+    }
+    id += kWarps / (2 * s);
+  }
+  return best;
+}
+
 // Merges the 8 warps' descending lists (`best` in each warp) into lists[0..31], pairwise in 3
 // levels. `lists` needs kWarps * 32 entries. Contains CTA barriers.
 __device__ __forceinline__ void cta_merge_warp_lists(uint64_t best, uint64_t* lists) {

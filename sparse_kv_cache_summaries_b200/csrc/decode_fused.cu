@@ -94,7 +94,7 @@ struct FLay {
     pw = o;     o = a16(o + sizeof(float) * G * kRound);
     sc = o;     o = a16(o + sizeof(float) * 8);
     fac = o;    o = a16(o + sizeof(float) * G * 34);
-    mbar = o;   o = a16(o + 8 * 2);
+    mbar = o;   o = a16(o + 8 * 3);
     total = o;
   }
 };
@@ -199,10 +199,32 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   float* fac_s = reinterpret_cast<float*>(sm + L.fac);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L.mbar);
 
-  // ---- prologue (inputs written before the streaming kernel started)
+  // Exchanges between the ranks are pushes: a rank writes into the receiver's shared memory with
+  // st.async, which completes bytes on the receiver's mbarrier, and the receiver waits (bounded)
+  // on its own mbarrier for exactly the bytes it expects:
+  //   mbar[0]  rank 0: the C candidate lists (warp Top-K path)
+  //   mbar[1]  this rank's selection slots, from rank 0 (warp Top-K path)
+  //   mbar[2]  merging ranks: the C partials of their output slice and (M, L) of its heads
+  constexpr int E = G * D;
+  const bool warp_topk = p.do_select && p.Kb > 0 && p.Kb <= kWarpTopK;
+  const int first_owner = (p.do_select && C > 1) ? 1 : 0;
+  const int n_owners = C - first_owner;
+  const int per_o = (E + n_owners - 1) / n_owners;
+  const int wr = rank - first_owner;                    // this rank's output slice, if >= 0
+  const int oe0 = wr >= 0 ? min(E, wr * per_o) : E, oe1 = wr >= 0 ? min(E, oe0 + per_o) : E;
+  const int per_slot = (p.Kb + C - 1) / C;
+  const int my_slots = max(0, min(per_slot, p.Kb - rank * per_slot));
   if (tid == 0) {
-    mbar_init(&mbar[1], 1);  // this rank's selection slots, delivered by rank 0
+    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[1], 1);
+    mbar_init(&mbar[2], 1);
     mbar_init_fence();
+    if (warp_topk && rank == 0) mbar_arrive_expect_tx(&mbar[0], static_cast<uint32_t>(C * 32 * 8));
+    if (warp_topk && p.do_attend && my_slots > 0) mbar_arrive_expect_tx(&mbar[1], static_cast<uint32_t>(my_slots * 4));
+    if (p.do_attend && oe0 < oe1) {
+      const int nh = (oe1 - 1) / D - oe0 / D + 1;
+      mbar_arrive_expect_tx(&mbar[2], static_cast<uint32_t>(C * ((oe1 - oe0) * 4 + nh * 8)));
+    }
   }
   if (p.do_attend) {
     const T* qp = static_cast<const T*>(p.q) + static_cast<size_t>(pr) * G * D;
@@ -264,7 +286,6 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     float lz[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) lz[h] = logz[h];
-    const bool warp_topk = Kb > 0 && Kb <= kWarpTopK;
     // S_j of chunk k of this warp, as a key (empty blocks: 0); also written to `scores`
     auto key_of = [&](int k, int j) -> uint32_t {
       if (j >= nloc) return 0u;
@@ -285,10 +306,11 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       return empty ? 0u : score_key(S);
     };
     if (tid == 0) misc[0] = 0;
+    uint64_t best = 0ull;  // warp 0 ends with this rank's best-32 list (warp Top-K path)
     if (warp_topk) {
       // this rank's best 32 (descending codes) in hist[0..255]: a superset of its share. Chunks
       // go in pairs: two independent sorts, then one merge.
-      uint64_t best = 0ull;
+      best = 0ull;
       for (int k = 0; k * 32 < span; k += 2) {
         const int ja = jb + k * 32 + lane, jc = ja + 32;
         const uint32_t ka = key_of(k, ja);
@@ -298,12 +320,12 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         const uint64_t m2 = warp_merge_top32(sa, sc);
         best = (k == 0) ? m2 : warp_merge_top32(best, m2);
       }
-      cta_merge_warp_lists(best, reinterpret_cast<uint64_t*>(hist));
+      best = warp_pairs_merge_top32(best, reinterpret_cast<uint64_t*>(hist));  // warp 0: the rank's list
       if (p.do_attend && warp == 0) {
         // speculative: this rank's likeliest picks start moving from HBM to L2 while the global
         // cut runs (about 2 K_b / C of them: the global Top-K_b holds K_b / C per rank on average)
         const int m = min(32, max(1, (2 * Kb + C - 1) / C));
-        const uint64_t code = reinterpret_cast<const uint64_t*>(hist)[lane];
+        const uint64_t code = best;
         if (lane < m && code != 0ull) {
           const int j = topk_index(code);
           const size_t off = (static_cast<size_t>(pr) * p.T + static_cast<size_t>(j) * kBlockTokens) * D;
@@ -339,16 +361,18 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       }
     }
     cluster_wait();  // every rank has started: peers' shared memory may be written
-    if (warp_topk && warp == 0) {  // push this rank's list to rank 0
-      const uint64_t code = reinterpret_cast<const uint64_t*>(hist)[lane];
-      *cluster.map_shared_rank(reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + rank * 32 + lane, 0) = code;
+    if (warp_topk && warp == 0) {  // push this rank's list into rank 0
+      const uint64_t code = best;
+      st_async_b64(cluster_smem_addr(reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + rank * 32 + lane, 0), code,
+                   cluster_smem_addr(&mbar[0], 0));
     }
-    cluster.sync();  // #1: every rank's candidates are visible
+    if (!warp_topk) cluster.sync();  // #1 (radix path): every rank's candidates are visible
 
     // ---- 2. rank 0: global Top-K_b from the ranks' candidates; other ranks: compensation merge
     if (rank == 0 && Kb > 0 && Kb <= kWarpTopK) {
       // merge the C ranks' best-32 lists pairwise (the first level straight from the ranks'
       // shared memory), then order the first K_b by block index
+      mbar_wait_cluster(&mbar[0], 0, p.status);  // the C lists have arrived
       const uint64_t* rl = reinterpret_cast<const uint64_t*>(hist) + kWarps * 32;  // [C][32] pushed
       uint64_t* g0 = reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + kMaxCluster * 32;
       uint64_t* g1 = g0 + kWarps * 32;
@@ -375,15 +399,15 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         const int idx = warp_sort_asc(lane < Kb ? topk_index(src[lane]) : 0x7fffffff);
         if (lane < Kb && p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + lane] = idx;
         if (p.do_attend) {
-          // lane r writes rank r's slots [r per, r per + per) into its shared memory, then
-          // releases them to it with a remote arrive: rank r starts at once, no cluster barrier
-          const int per = (Kb + C - 1) / C;
-          for (int q = 0; q < per; ++q) {
-            const int slot = lane * per + q;
+          // lane r pushes rank r's slots [r per, r per + per) into its shared memory; rank r
+          // starts as soon as its bytes land, with no cluster barrier
+          for (int q = 0; q < per_slot; ++q) {
+            const int slot = lane * per_slot + q;
             const int v = __shfl_sync(0xffffffffu, idx, slot < 32 ? slot : 0);
-            if (lane < C && slot < Kb) *cluster.map_shared_rank(&selm[q], lane) = v;
+            if (lane < C && slot < Kb)
+              st_async_b32(cluster_smem_addr(&selm[q], lane), static_cast<uint32_t>(v),
+                           cluster_smem_addr(&mbar[1], lane));
           }
-          if (lane < C) mbar_arrive_remote(cluster_smem_addr(&mbar[1], lane));
         }
         if (lane == 0) misc[6] = Kb;
       }
@@ -473,13 +497,11 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       o[0] = cM[tid];
       o[1] = cl[tid];
     }
-    if (!warp_topk) cluster.sync();  // #2: the cut is visible (radix path; the warp path
-                                      // delivers the slots through mbar[1])
+    if (!warp_topk) cluster.sync();  // #2 (radix path): the cut is visible
 
     // ---- 3a. this rank's share of the selection: a contiguous slice of rank 0's ordered list
-    if (p.do_attend && warp_topk) {  // rank 0 delivers this rank's slots
-      const int per = (Kb + C - 1) / C;
-      nsel = mbar_wait_cluster(&mbar[1], 0, p.status) ? max(0, min(per, Kb - rank * per)) : 0;
+    if (p.do_attend && warp_topk) {  // rank 0 pushes this rank's slots
+      nsel = (my_slots == 0 || __syncthreads_and(mbar_wait_cluster(&mbar[1], 0, p.status))) ? my_slots : 0;
     } else if (p.do_attend && Kb > 0) {
       const int total = *cluster.map_shared_rank(&misc[6], 0);
       const int per = (total + C - 1) / C;
@@ -498,7 +520,10 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     nsel = s1 - s0;
     __syncthreads();
   }
-  if (!p.do_attend) return;  // select only: no rank touches another's shared memory from here
+  if (!p.do_attend) {  // select only: no CTA leaves while a peer's push into it may be in flight
+    cluster.sync();
+    return;
+  }
 
   // ---- 3b. exact attention over this rank's selected blocks. Work unit: a group of 4 rows of
   // one block; warp w takes groups w, w + 8, ... Each lane holds VEP = D / 32 channels of every
@@ -642,29 +667,27 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   float* wf = wml + kWarps * G * 2;  // [kWarps][G] factors
   float* rM = wf + kWarps * G;       // [G] this rank's reference per head
   float* rL = rM + G;                // [G]
-  if (tid < G) {
-    const int h = tid;
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wml[(w * G + h) * 2]);
-    float Lsum = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float mwv = wml[(w * G + h) * 2];
-      const float f = (mwv == -CUDART_INF_F) ? 0.f : __expf(mwv - M);
-      wf[w * G + h] = f;
-      Lsum = fmaf(f, wml[(w * G + h) * 2 + 1], Lsum);
+  if (warp < G) {  // warp h: head h's factors over the 8 warps (lanes 0..7, butterflies of 8)
+    const int h = warp;
+    const float mwv = lane < kWarps ? wml[(lane * G + h) * 2] : -CUDART_INF_F;
+    float M = mwv;
+#pragma unroll
+    for (int o = kWarps / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float f = (mwv == -CUDART_INF_F) ? 0.f : __expf(mwv - M);
+    float Lsum = lane < kWarps ? f * wml[(lane * G + h) * 2 + 1] : 0.f;
+#pragma unroll
+    for (int o = kWarps / 2; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    if (lane < kWarps) wf[lane * G + h] = f;
+    if (lane == 0) {
+      rM[h] = M;
+      rL[h] = Lsum;
     }
-    rM[h] = M;
-    rL[h] = Lsum;
   }
   __syncthreads();
   // ---- this rank's partial, pushed to the ranks that merge the outputs. Output channels
   // [0, E) are cut into slices, one per merging rank: with selection ranks 1..C-1 (each holds
   // the compensation sum of its slice), without it ranks 0..C-1 (C = 1: rank 0 alone). Every
   // rank writes its partial of a slice into the merging rank's receive buffers.
-  constexpr int E = G * D;
-  const int first_owner = (p.do_select && C > 1) ? 1 : 0;
-  const int n_owners = C - first_owner;
-  const int per_o = (E + n_owners - 1) / n_owners;
   float* racc = acc_s;  // [C][per_o] received partial sums
   float* rml = ml_s;    // [C][G][2] received (M, L)
   if (!p.do_select) cluster_wait();  // every rank has started: peers may be written
@@ -673,9 +696,8 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     const int o_lo = first_owner + (h * D) / per_o, o_hi = first_owner + (h * D + D - 1) / per_o;
     const int o = o_lo + lane;
     if (o <= o_hi) {
-      float* dst = cluster.map_shared_rank(rml + (rank * G + h) * 2, o);
-      dst[0] = rM[h];
-      dst[1] = rL[h];
+      const uint64_t ml = (static_cast<uint64_t>(__float_as_uint(rL[h])) << 32) | __float_as_uint(rM[h]);
+      st_async_b64(cluster_smem_addr(rml + (rank * G + h) * 2, o), ml, cluster_smem_addr(&mbar[2], o));
     }
   }
   for (int i = tid; i < E; i += kThreads) {
@@ -684,14 +706,16 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) a = fmaf(wf[w * G + h], wacc[w * E + i], a);
     const int ow = i / per_o;
-    *cluster.map_shared_rank(racc + rank * per_o + (i - ow * per_o), first_owner + ow) = a;
+    st_async_b32(cluster_smem_addr(racc + rank * per_o + (i - ow * per_o), first_owner + ow), __float_as_uint(a),
+                 cluster_smem_addr(&mbar[2], first_owner + ow));
   }
-  cluster.sync();  // #3: every partial pushed to this rank is visible
+  cluster_arrive();  // this rank's pushes are issued (matched by the wait before exit)
 
   // ---- 4. outputs of this rank's slice, from its receive buffers (local reads only)
-  const int wr = rank - first_owner;
-  if (wr >= 0) {
-    const int e0 = min(E, wr * per_o), e1 = min(E, e0 + per_o);
+  bool have = false;  // uniform over the CTA (a wait that gave up in any thread skips the merge)
+  if (wr >= 0 && oe0 < oe1) have = __syncthreads_and(mbar_wait_cluster(&mbar[2], 0, p.status)) != 0;
+  if (have) {
+    const int e0 = oe0, e1 = oe1;
     const float* cpg = p.comp + static_cast<size_t>(pr) * G * (D + 2);
     if (e0 < e1) {
       const int hlo = e0 / D, nh = (e1 - 1) / D - hlo + 1;
@@ -725,6 +749,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       }
     }
   }
+  cluster_wait();  // no CTA leaves while a peer's push into it may be in flight
 }
 
 template <typename T, int D, typename S>
