@@ -234,6 +234,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   cluster_arrive_relaxed();  // matched by cluster_wait() before this CTA first writes a peer
 
   pdl_wait();  // the previous kernel's outputs are visible from here on
+  pdl_launch_dependents();  // every CTA of this grid is resident: the next grid may stage in
 
   const int Kb = p.Kb;
   const int j0 = rank * p.chunk;

@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   }
   if (tid < 17) logn_s[tid] = tid > 0 ? logf(static_cast<float>(tid)) : -CUDART_INF_F;
   __syncthreads();
+  // Launched with programmatic serialisation: everything above touches shared memory only, so it
+  // overlaps the previous kernel's tail; every global read and write comes after this wait.
+  pdl_wait();
   // (pair, tile within the pair) of tile k + d, from those of tile k
   auto advance = [&](int pr, int t, int d, int& pr_out, int& t_out) {
     t += d;
@@ -607,7 +610,11 @@ cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = g.smem;
   cfg.stream = st;
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   void* args[] = {&p};
   return cudaLaunchKernelExC(&cfg, kern, args);
 }
