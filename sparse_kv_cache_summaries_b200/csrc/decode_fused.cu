@@ -21,16 +21,16 @@
 //     kv-head's segments, a slice of channels each.
 //  3. Rank c attends the c-th contiguous slice of rank 0's ordered selection (balanced whatever
 //     the blocks' positions; rank 0 writes each rank's slots into its shared memory and releases
-//     them with a remote mbarrier arrive): bulk copies of their K and V rows (up to the
-//     cache capacity; rows past the block's token count are masked) and of their mean values,
-//     exact logits, an online softmax per head, P.V, and removal of the blocks' compensation terms
-//     (taken against the running max of the exact logits, which is at least every processed
-//     block's mean logit, so nothing overflows; a block's compensation mass never exceeds its
-//     exact mass, so the removal cancels at most what it adds).
+//     them through st.async bytes counted on the rank's mbarrier): their K and V rows read
+//     straight into registers (up to the cache capacity; rows past the block's token count are
+//     masked) with the blocks' mean values, exact logits, an online softmax per warp and head,
+//     P.V, and removal of the blocks' compensation terms (taken against a reference at least
+//     every processed block's mean logit, so nothing overflows; a block's compensation mass
+//     never exceeds its exact mass, so the removal cancels at most what it adds).
 //  4. Every rank pushes its partial of each output slice into the rank that merges the slice
-//     (distributed shared memory stores); after one cluster barrier each merging rank combines
-//     its slice from local memory with the compensation partial (with selection, the slice whose
-//     compensation sum it merged).
+//     (st.async into the receiver's shared memory, counted on its mbarrier); each merging rank
+//     combines its slice from local memory with the compensation partial (with selection, the
+//     slice whose compensation sum it merged).
 // Flags run steps 1-2 only (score/select call) or steps 3-4 only on a given selection (sparse
 // decode call). Launched with programmatic dependent launch: the prologue overlaps the previous
 // kernel's tail.
@@ -48,8 +48,6 @@ namespace compkv {
 namespace {
 
 constexpr int kMaxCluster = 16;
-constexpr int kRound = 8;  // selected blocks per shared-memory round
-constexpr int kRows = kRound * kBlockTokens;
 constexpr int kWarpTopK = 32;  // K_b up to this: warp bitonic Top-K; above: radix select
 
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
@@ -58,8 +56,8 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast
 struct FLay {
   int chunk, ccap, gcap, slots;
   size_t keys, ck, ci, gk, gi, hist, bc, sh, misc, zm, zs, fm, fl, cslice, selm;
-  size_t q, kbuf, vbuf, nu, lg, pT, red, acc, ml, blk, xr, pw, sc, fac, mbar, total;
-  __host__ __device__ void build(int chunk_, int Kb, int C, int slots_, int G, int D, int esz, int ksub) {
+  size_t q, wacc, wml, red, acc, ml, sc, fac, mbar, total;
+  __host__ __device__ void build(int chunk_, int Kb, int C, int slots_, int G, int D) {
     chunk = chunk_;
     slots = slots_;
     ccap = Kb < chunk ? Kb : chunk;
@@ -81,17 +79,11 @@ struct FLay {
     cslice = o; o = a16(o + sizeof(float) * G * D);
     selm = o;   o = a16(o + sizeof(int) * (Kb + 1));
     q = o;      o = a16(o + sizeof(float) * G * D);
-    kbuf = o;   o = a16(o + static_cast<size_t>(esz) * kRows * D);
-    vbuf = o;   o = a16(o + static_cast<size_t>(esz) * kRows * D);
-    nu = o;     o = a16(o + sizeof(float) * kRound * D);
-    lg = o;     o = a16(o + sizeof(float) * G * kRows);
-    pT = o;     o = a16(o + sizeof(float) * G * kRows);
-    red = o;    o = a16(o + sizeof(float) * (ksub * G * D > 256 ? ksub * G * D : 256));
+    wacc = o;   o = a16(o + sizeof(float) * kWarps * G * D);      // the warps' partial sums
+    wml = o;    o = a16(o + sizeof(float) * (3 * kWarps * G + 2 * G));  // (M, L), factors, rank's
+    red = o;    o = a16(o + sizeof(float) * 256);                    // compensation merge scratch
     acc = o;    o = a16(o + sizeof(float) * 2 * G * D);          // received partials [C][slice]
     ml = o;     o = a16(o + sizeof(float) * kMaxCluster * 2 * G);  // received (m, l) [C][G][2]
-    blk = o;    o = a16(o + sizeof(int) * 2 * kRound);
-    xr = o;     o = a16(o + sizeof(float) * G * kRound);
-    pw = o;     o = a16(o + sizeof(float) * G * kRound);
     sc = o;     o = a16(o + sizeof(float) * 8);
     fac = o;    o = a16(o + sizeof(float) * G * 34);
     mbar = o;   o = a16(o + 8 * 3);
@@ -154,6 +146,28 @@ struct RowPart {
   }
 };
 
+// The G log scores of one block (G consecutive floats, aligned to G floats) as vector loads.
+template <int G>
+__device__ __forceinline__ void load_scores(const float* src, float (&d)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G / 4; ++i) {
+      const float4 t = reinterpret_cast<const float4*>(src)[i];
+      d[4 * i] = t.x;
+      d[4 * i + 1] = t.y;
+      d[4 * i + 2] = t.z;
+      d[4 * i + 3] = t.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(src);
+    d[0] = t.x;
+    d[1] = t.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < G; ++i) d[i] = src[i];
+  }
+}
+
 __device__ __forceinline__ int stream_cta_of_tile(long long f, int nctas, int F) {
   return static_cast<int>(((f + 1) * nctas - 1) / F);
 }
@@ -190,8 +204,6 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   float* cslice = reinterpret_cast<float*>(sm + L.cslice);
   int* selm = reinterpret_cast<int*>(sm + L.selm);
   float* q_s = reinterpret_cast<float*>(sm + L.q);
-  T* kbuf = reinterpret_cast<T*>(sm + L.kbuf);
-  float* lg_s = reinterpret_cast<float*>(sm + L.lg);
   float* red = reinterpret_cast<float*>(sm + L.red);
   float* acc_s = reinterpret_cast<float*>(sm + L.acc);
   float* ml_s = reinterpret_cast<float*>(sm + L.ml);
@@ -266,7 +278,8 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     for (int k = 0; k < UPT; ++k) {
       const int j = jb + k * 32 + lane;
 #pragma unroll
-      for (int h = 0; h < G; ++h) ur[k][h] = (k * 32 < span && j < nloc) ? up[static_cast<size_t>(j) * G + h] : 0.f;
+      for (int h = 0; h < G; ++h) ur[k][h] = 0.f;
+      if (k * 32 < span && j < nloc) load_scores<G>(up + static_cast<size_t>(j) * G, ur[k]);
     }
     __syncthreads();
     // ---- 1b. log Zhat per head; compensation max, factors and sum per head
@@ -299,8 +312,10 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
             for (int h = 0; h < G; ++h) S += __expf(ur[kk][h] - lz[h]);
           }
       } else {
+        float uj[G];
+        load_scores<G>(up + static_cast<size_t>(j) * G, uj);
 #pragma unroll
-        for (int h = 0; h < G; ++h) S += __expf(up[static_cast<size_t>(j) * G + h] - lz[h]);
+        for (int h = 0; h < G; ++h) S += __expf(uj[h] - lz[h]);
       }
       const bool empty = S != S;
       if (p.scores) p.scores[static_cast<size_t>(pr) * p.Nb + j0 + j] = empty ? 0.f : S;
@@ -650,8 +665,8 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   }
 
   // ---- the warps' partials -> this rank's partial (M_h, L_h, A_h) in shared memory
-  float* wacc = reinterpret_cast<float*>(kbuf);  // [kWarps][G][D]
-  float* wml = lg_s;                             // [kWarps][G][2], then factors [kWarps][G]
+  float* wacc = reinterpret_cast<float*>(sm + L.wacc);  // [kWarps][G][D]
+  float* wml = reinterpret_cast<float*>(sm + L.wml);    // [kWarps][G][2], then factors [kWarps][G]
 #pragma unroll
   for (int h = 0; h < G; ++h) {
 #pragma unroll
@@ -764,7 +779,6 @@ const void* kptr_g(int G) {
   return nullptr;
 }
 
-int ksub_of(bool bf16, int D) { return kThreads / (D / (bf16 ? 2 : 1)); }
 
 template <typename S>
 const void* pick_s(bool bf16, int D, int G) {
@@ -813,11 +827,10 @@ cudaError_t make_plan(const void* kern, const FusedArgs& a, Plan* out) {
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   int C0 = 1;
   while (C0 < kMaxCluster && a.pairs * (2 * C0) <= 2 * sms && (a.Nb + 2 * C0 - 1) / (2 * C0) >= 64) C0 *= 2;
-  const int esz = a.bf16 ? 2 : 4;
   for (int C = C0; C >= 1; C /= 2) {
     const int chunk = (a.Nb + C - 1) / C;
     FLay L;
-    L.build(chunk, a.Kb, C, a.slots, a.G, a.D, esz, ksub_of(a.bf16, a.D));
+    L.build(chunk, a.Kb, C, a.slots, a.G, a.D);
     if (L.total > static_cast<size_t>(optin)) continue;
     // the opt-in maximum, so that plans of different sizes share the kernel's attribute
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
