@@ -13,11 +13,11 @@
 // bytes whatever B and Hkv are. A CTA's range crosses at most a few (sequence, kv-head) pairs; it
 // writes one partial record per pair it touches ("segment").
 //
-// Pipeline: a 3-stage shared-memory ring with a "full" mbarrier per stage. Each warp releases a
-// stage by bumping a shared counter; the last of the 8 to release it refills it at once (bulk
-// copies of the tile's mean keys and mean values, 4-byte cp.async of its grouped variances and
-// counts), so no warp waits to produce. Each warp owns 4 blocks of every tile and works through
-// the ring on its own, with no CTA barrier in steady state. Lane l holds the same VW channels of
+// Pipeline: a 3-stage shared-memory ring with a "full" and an "empty" mbarrier per stage. A
+// producer warp fills the stages (bulk copies of the tile's mean keys and mean values, 4-byte
+// cp.async of its grouped variances and counts) as soon as the 8 consumer warps have released
+// them, so no consumer ever pays for issuing a copy. Each consumer warp owns 4 blocks of every
+// tile and works through the ring on its own, with no CTA barrier in steady state. Lane l holds the same VW channels of
 // every row for all G heads, so each mean key and mean value is read from shared memory once:
 // partial dots of the 4 blocks with the G heads, one transpose-reduce over the warp that leaves
 // each lane with one (block, head) dot for the scalar work, then each lane accumulates its
@@ -39,7 +39,9 @@ namespace {
 
 constexpr int kTile = kStreamTile;
 constexpr int kStages = 3;
-constexpr int kBlocksPerWarp = kTile / kWarps;  // 4
+constexpr int kBlocksPerWarp = kTile / kWarps;  // 4 (kWarps consumer warps)
+constexpr int kStreamThreads = (kWarps + 1) * 32;  // the consumers and one producer warp
+constexpr int kConsumerBar = 1;                    // named barrier of the consumer warps
 constexpr float kRefSlack = 64.f;
 
 struct StreamParams {
@@ -71,8 +73,8 @@ struct SLay {
     const size_t scratch = sizeof(float) * kWarps * G * D;
     if (stage_bytes < scratch) stage_bytes = a16(scratch);
     size_t o = 0;
-    full = o;   o = a16(o + 8 * kStages);
-    rel = o;    o = a16(o + sizeof(uint32_t) * (kStages + 2));  // release counters, abort, issued
+    full = o;   o = a16(o + 8 * 2 * kStages);                   // full[kStages], empty[kStages]
+    rel = o;    o = a16(o + sizeof(uint32_t) * 4);              // abort flag
     wsw = o;    o = a16(o + sizeof(float) * kWarps * kBlocksPerWarp * G);   // per-warp weights
     stage0 = o; o = a16(o + stage_bytes * kStages);
     q = o;      o = a16(o + sizeof(float) * G * D);
@@ -109,7 +111,7 @@ __device__ __forceinline__ void row_pairs(const S* row, float2 (&a)[VW / 2]) {
 
 // S: storage type of the mean key and mean value (float, or __half).
 template <typename TQ, int D, int G, int R, typename S>
-__global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_constant__ StreamParams p) {
+__global__ void __launch_bounds__(kStreamThreads, 2) score_stream_kernel(const __grid_constant__ StreamParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   SLay L;
   L.build(D, G, p.r, sizeof(S));
@@ -122,10 +124,9 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   const int nt = f1 - f0;
   constexpr int XS = xrec_stride(G);
 
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.full);
-  uint32_t* rel_s = reinterpret_cast<uint32_t*>(sm + L.rel);  // [kStages] warps released, ever
-  volatile uint32_t* abort_s = rel_s + kStages;                // a wait gave up: issue no more
-  uint32_t* issued_s = rel_s + kStages + 1;                    // tiles issued so far
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.full);  // [kStages]: the tile has landed
+  uint64_t* empty = full + kStages;                            // [kStages]: the 8 warps are done
+  volatile uint32_t* abort_s = reinterpret_cast<uint32_t*>(sm + L.rel);  // a wait gave up
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   float* qn_s = reinterpret_cast<float*>(sm + L.qn);
   float* refw_s = reinterpret_cast<float*>(sm + L.refw);
@@ -156,11 +157,10 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 32 + 1);
-      rel_s[s] = 0;
+      mbar_init(&full[s], 32 + 1);   // the producer's 32 lanes (cp.async) + the byte count
+      mbar_init(&empty[s], kWarps);  // one arrival per consumer warp
     }
     *abort_s = 0;
-    *issued_s = min(nt, kStages);
     mbar_init_fence();
   }
   if (tid < 17) logn_s[tid] = tid > 0 ? logf(static_cast<float>(tid)) : -CUDART_INF_F;
@@ -168,24 +168,37 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   // Launched with programmatic serialisation: everything above touches shared memory only, so it
   // overlaps the previous kernel's tail; every global read and write comes after this wait.
   pdl_wait();
-  // (pair, tile within the pair) of tile k + d, from those of tile k
-  auto advance = [&](int pr, int t, int d, int& pr_out, int& t_out) {
-    t += d;
-    while (t >= TP) {
-      t -= TP;
-      ++pr;
-    }
-    pr_out = pr;
-    t_out = t;
-  };
   const int pr0 = f0 / TP, t0 = f0 % TP;
-  if (warp == 0)
-    for (int k = 0; k < min(nt, kStages); ++k) {
-      int pk, tk;
-      advance(pr0, t0, k, pk, tk);
-      issue(k, pk, tk);
-    }
   pdl_launch_dependents();
+
+  if (warp == kWarps) {
+    // ---- producer: tile k goes into stage k % kStages once the consumer warps have released
+    // tile k - kStages (the k / kStages - 1 th completion of that stage's empty barrier)
+    int pr = pr0, tt = t0, issued = 0;
+    for (int k = 0; k < nt; ++k) {
+      const int st = k % kStages;
+      if (k >= kStages) {
+        bool got = mbar_wait(&empty[st], static_cast<uint32_t>((k / kStages - 1) & 1), p.status);
+        got = __all_sync(0xffffffffu, got);
+        if (!got && lane == 0) *abort_s = 1;
+        if (!got || *abort_s != 0) break;
+        // the consumers' generic-proxy reads (and merge scratch writes) of the stage come first
+        fence_proxy_async();
+      }
+      issue(k, pr, tt);
+      ++issued;
+      if (++tt == TP) {
+        tt = 0;
+        ++pr;
+      }
+    }
+    if (*abort_s != 0) {  // a wait gave up (status recorded): wait, bounded, for the copies in flight
+      for (int k = max(0, issued - kStages); k < issued; ++k)
+        mbar_wait(&full[k % kStages], static_cast<uint32_t>((k / kStages) & 1), nullptr);
+    }
+    __syncthreads();  // matched by the consumers' barrier after their loop: no copy is in flight
+    return;
+  }
 
   // Lane map: lane l holds channels [l VW, l VW + VW) of every row for all G heads (a warp-wide
   // row load is one contiguous 512 or 256 bytes: each mean key and mean value is read from
@@ -209,8 +222,11 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   int cur = -1;
   float* wsw = reinterpret_cast<float*>(sm + L.wsw) + warp * NVAL;  // weights of the warp's pairs
 
-  // Merges the 8 warps' partials of the current segment (pair `cur`) in a fixed order, with the
+  // Merges the 8 consumer warps' partials of the current segment (pair `cur`) in a fixed order, with the
   // stage `free_stage` (no copy in flight) as scratch for the warps' weighted mean-value sums.
+  // the consumer warps' CTA barrier (the producer warp takes no part)
+  auto consumer_sync = [&]() { named_bar_sync(kConsumerBar, kWarps * 32); };
+
   auto finish_segment = [&](int free_stage) {
     if (lane == 0) {
 #pragma unroll
@@ -220,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       red_s[(0 * G + my_h) * 32 + slot] = zmax;
       red_s[(1 * G + my_h) * 32 + slot] = zsum;
     }
-    __syncthreads();
+    consumer_sync();
     float fw[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -246,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
         }
       }
     }
-    __syncthreads();
+    consumer_sync();
     const int k = blockIdx.x - static_cast<int>(((static_cast<long long>(cur) * TP + 1) * p.nctas - 1) / F);
     const size_t rec = static_cast<size_t>(cur) * p.slots + k;
     if (warp < G) {  // warp hh: head hh's 32 slots, butterfly merges (fixed order)
@@ -279,14 +295,14 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
         p.comp[(rec * G + i / D) * (D + 2) + 2 + (i % D)] = v;
       }
     }
-    __syncthreads();  // the scratch stage and the slots are free again
+    consumer_sync();  // the scratch stage and the slots are free again
   };
 
   // Loads the query heads of pair `pr` and resets the running state.
   auto start_segment = [&](int pr) {
     const TQ* qp = static_cast<const TQ*>(p.q) + static_cast<size_t>(pr) * G * D;
     for (int i = tid; i < G * D; i += kThreads) q_s[i] = to_float(qp[i]);
-    __syncthreads();
+    consumer_sync();
     const int gsz = D / r;
     for (int i = tid; i < G * r; i += kThreads) {
       const int hh = i / r, g = i % r;
@@ -297,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       }
       qn_s[i] = p.scale * p.scale * s;
     }
-    __syncthreads();
+    consumer_sync();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float* qh = q_s + h * D + lane * VW;
@@ -314,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
     }
     zmax = -CUDART_INF_F;
     zsum = lsum = 0.f;
-    __syncthreads();
+    consumer_sync();
   };
 
   // `ok` goes false (for this warp) once a wait gives up; the warp then stops waiting and
@@ -324,18 +340,13 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
   int st = 0, ph = 0;         // ring stage and its phase parity for tile k
 #pragma unroll 1
   for (int k = 0; k < nt; ++k) {
-    if (pr != cur) {  // every warp reaches this at the same tile
-      __syncthreads();
-      // the stage of tile k - 1 is free: its refill waits until this segment switch is done
+    if (pr != cur) {  // every consumer warp reaches this at the same tile
+      consumer_sync();
+      // the stage of tile k - 1 (not yet released) is the merge's scratch; released afterwards
       if (cur >= 0) finish_segment((k + kStages - 1) % kStages);
       start_segment(pr);
       cur = pr;
-      if (warp == 0 && k >= 1 && k + kStages - 1 < nt && *abort_s == 0) {
-        int pk, tk;
-        advance(pr, tt, kStages - 1, pk, tk);
-        issue(k + kStages - 1, pk, tk);
-        if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(k + kStages));
-      }
+      if (k >= 1 && lane == 0) mbar_arrive(&empty[(k + kStages - 1) % kStages]);
     }
     bool got = ok && mbar_wait(&full[st], ph, p.status);
     got = __all_sync(0xffffffffu, got);
@@ -460,26 +471,10 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       }
     }
 
-    // release the stage; the last of the 8 warps to do so refills it with tile k + kStages
-    // (unless tile k + 1 starts a new segment: then the refill waits for the segment switch)
+    // release the stage to the producer (unless tile k + 1 starts a new segment: the stage is
+    // then the segment merge's scratch and is released after it)
     __syncwarp();
-    uint32_t before = 0;
-    if (lane == 0) {
-      __threadfence_block();
-      before = atomicAdd(&rel_s[st], 1u);
-    }
-    before = __shfl_sync(0xffffffffu, before, 0);
-    if (before % kWarps == kWarps - 1) {
-      const int kk = k + kStages;
-      const bool defer = k + 1 < nt && tt + 1 == TP;
-      if (kk < nt && !defer && *abort_s == 0) {
-        fence_proxy_async();
-        int pk, tk;
-        advance(pr, tt, kStages, pk, tk);
-        issue(kk, pk, tk);
-        if (lane == 0) atomicMax(issued_s, static_cast<uint32_t>(kk + 1));
-      }
-    }
+    if (lane == 0 && !(k + 1 < nt && tt + 1 == TP)) mbar_arrive(&empty[st]);
     if (rep && jm < tn) {
       const size_t row = static_cast<size_t>(pr) * p.Nb + jt0 + jm;
       p.u[row * G + my_h] = st_u;
@@ -495,13 +490,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_stream_kernel(const __grid_
       ph ^= 1;
     }
   }
-  __syncthreads();
-  if (*abort_s != 0 && warp == 0) {
-    // a wait gave up (status recorded): wait, bounded, for the copies still in flight
-    const int n_iss = static_cast<int>(*issued_s);
-    for (int k = max(0, n_iss - kStages); k < n_iss; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, nullptr);
-  }
-  __syncthreads();
+  __syncthreads();  // with the producer, which has drained any copy still in flight
   if (cur >= 0) finish_segment(0);
 }
 
@@ -561,7 +550,7 @@ cudaError_t grid_for(const void* kern, int D, int G, int r, bool fp16, Grid* out
   g.smem = L.total;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(g.smem));
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&g.ctas_per_sm, kern, kThreads, g.smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&g.ctas_per_sm, kern, kStreamThreads, g.smem);
   if (e != cudaSuccess) return e;
   if (g.ctas_per_sm < 1) return cudaErrorInvalidConfiguration;
   cudaDeviceGetAttribute(&g.sms, cudaDevAttrMultiProcessorCount, dev);
@@ -607,7 +596,7 @@ cudaError_t launch_score_stream(const StreamArgs& a, cudaStream_t st) {
   if (a.nctas_out) *a.nctas_out = p.nctas;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.nctas, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kStreamThreads, 1, 1);
   cfg.dynamicSmemBytes = g.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
