@@ -220,14 +220,18 @@ __global__ void __launch_bounds__(kStreamThreads, 2) score_stream_kernel(const _
   float mref[G];          // this warp's reference logit per head
   float zmax = -CUDART_INF_F, zsum = 0.f, lsum = 0.f;  // this lane's (block, head) partials
   int cur = -1;
+  size_t seg_rec = 0;  // record index of the current segment
   float* wsw = reinterpret_cast<float*>(sm + L.wsw) + warp * NVAL;  // weights of the warp's pairs
 
-  // Merges the 8 consumer warps' partials of the current segment (pair `cur`) in a fixed order, with the
-  // stage `free_stage` (no copy in flight) as scratch for the warps' weighted mean-value sums.
   // the consumer warps' CTA barrier (the producer warp takes no part)
   auto consumer_sync = [&]() { named_bar_sync(kConsumerBar, kWarps * 32); };
 
+  // Merges the 8 consumer warps' partials of the current segment (pair `cur`) in a fixed order,
+  // with the stage `free_stage` (no copy in flight) as scratch for the warps' mean-value sums.
   auto finish_segment = [&](int free_stage) {
+    // (1) each warp publishes its references, its slots' partials and its unscaled
+    // compensation sums (the stage `free_stage` is the scratch: [kWarps][G][D])
+    float* part = reinterpret_cast<float*>(sm + L.stage0 + L.stage_bytes * free_stage);
     if (lane == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) refw_s[warp * G + h] = mref[h];
@@ -235,64 +239,55 @@ __global__ void __launch_bounds__(kStreamThreads, 2) score_stream_kernel(const _
     if (rep) {
       red_s[(0 * G + my_h) * 32 + slot] = zmax;
       red_s[(1 * G + my_h) * 32 + slot] = zsum;
+      red_s[(2 * G + my_h) * 32 + slot] = lsum;
     }
-    consumer_sync();
-    float fw[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float M = -CUDART_INF_F;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, refw_s[w * G + h]);
-      fw[h] = (mref[h] == -CUDART_INF_F) ? 0.f : __expf(mref[h] - M);
-    }
-    float fme = fw[0];
-#pragma unroll
-    for (int h = 1; h < G; ++h) fme = (my_h == h) ? fw[h] : fme;
-    if (rep) red_s[(2 * G + my_h) * 32 + slot] = lsum * fme;
-    float* part = reinterpret_cast<float*>(sm + L.stage0 + L.stage_bytes * free_stage);  // [kWarps][G][D]
     if (compensate) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         float* pw = part + (warp * G + h) * D + lane * VW;
         if constexpr (VW == 4) {
-          reinterpret_cast<float4*>(pw)[0] =
-              make_float4(fw[h] * acc[h][0].x, fw[h] * acc[h][0].y, fw[h] * acc[h][1].x, fw[h] * acc[h][1].y);
+          reinterpret_cast<float4*>(pw)[0] = make_float4(acc[h][0].x, acc[h][0].y, acc[h][1].x, acc[h][1].y);
         } else {
-          reinterpret_cast<float2*>(pw)[0] = make_float2(fw[h] * acc[h][0].x, fw[h] * acc[h][0].y);
+          reinterpret_cast<float2*>(pw)[0] = acc[h][0];
         }
       }
     }
     consumer_sync();
-    const int k = blockIdx.x - static_cast<int>(((static_cast<long long>(cur) * TP + 1) * p.nctas - 1) / F);
-    const size_t rec = static_cast<size_t>(cur) * p.slots + k;
-    if (warp < G) {  // warp hh: head hh's 32 slots, butterfly merges (fixed order)
-      const int hh = warp;
-      float zm = red_s[(0 * G + hh) * 32 + lane], zs = red_s[(1 * G + hh) * 32 + lane];
-      float ls = red_s[(2 * G + hh) * 32 + lane];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, zm, o);
-        const float s2 = __shfl_xor_sync(0xffffffffu, zs, o);
-        lse_merge(zm, zs, m2, s2);
-        ls += __shfl_xor_sync(0xffffffffu, ls, o);
-      }
-      if (lane == 0) {
-        p.zpart[(rec * G + hh) * 2] = zm;
-        p.zpart[(rec * G + hh) * 2 + 1] = zs;
-        if (compensate) {
-          float Mh = -CUDART_INF_F;
-          for (int w = 0; w < kWarps; ++w) Mh = fmaxf(Mh, refw_s[w * G + hh]);
-          p.comp[(rec * G + hh) * (D + 2)] = Mh;
-          p.comp[(rec * G + hh) * (D + 2) + 1] = ls;
+    // (2) the per-head chains, spread over the warps (fixed order within each): chain c < G is
+    // head c's log-partition partial (max, then the sum rescaled to it); chain G + c is head c's
+    // compensation reference (the largest warp reference), the warps' rescale factors (written
+    // over their references) and the weight sum. Slot l belongs to warp l / kBlocksPerWarp.
+    for (int c = warp; c < 2 * G; c += kWarps) {
+      if (c < G) {
+        const float zm = red_s[(0 * G + c) * 32 + lane], zs = red_s[(1 * G + c) * 32 + lane];
+        const float M1 = warp_max(zm);
+        const float z = warp_sum(zm == -CUDART_INF_F ? 0.f : zs * __expf(zm - M1));
+        if (lane == 0) {
+          p.zpart[(seg_rec * G + c) * 2] = M1;
+          p.zpart[(seg_rec * G + c) * 2 + 1] = z;
+        }
+      } else if (compensate) {
+        const int h = c - G;
+        const float rw = lane < kWarps ? refw_s[lane * G + h] : -CUDART_INF_F;
+        const float Mh = warp_max(rw);
+        const float f = (rw == -CUDART_INF_F) ? 0.f : __expf(rw - Mh);
+        if (lane < kWarps) refw_s[lane * G + h] = f;
+        const float fl = __shfl_sync(0xffffffffu, f, lane / kBlocksPerWarp);
+        const float l = warp_sum(red_s[(2 * G + h) * 32 + lane] * fl);
+        if (lane == 0) {
+          p.comp[(seg_rec * G + h) * (D + 2)] = Mh;
+          p.comp[(seg_rec * G + h) * (D + 2) + 1] = l;
         }
       }
     }
-    if (compensate) {
+    if (compensate) {  // (3) the channels: sum over the warps of factor x partial
+      consumer_sync();
       for (int i = tid; i < G * D; i += kThreads) {
-        float v = part[i];
+        const int h = i / D;
+        float v = 0.f;
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) v += part[w * G * D + i];
-        p.comp[(rec * G + i / D) * (D + 2) + 2 + (i % D)] = v;
+        for (int w = 0; w < kWarps; ++w) v = fmaf(refw_s[w * G + h], part[w * G * D + i], v);
+        p.comp[(seg_rec * G + h) * (D + 2) + 2 + (i % D)] = v;
       }
     }
     consumer_sync();  // the scratch stage and the slots are free again
@@ -300,6 +295,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2) score_stream_kernel(const _
 
   // Loads the query heads of pair `pr` and resets the running state.
   auto start_segment = [&](int pr) {
+    // this CTA's record of pair pr: slot (this CTA - the first CTA whose range reaches pr)
+    seg_rec = static_cast<size_t>(pr) * p.slots + blockIdx.x -
+              static_cast<int>(((static_cast<long long>(pr) * TP + 1) * p.nctas - 1) / F);
     const TQ* qp = static_cast<const TQ*>(p.q) + static_cast<size_t>(pr) * G * D;
     for (int i = tid; i < G * D; i += kThreads) q_s[i] = to_float(qp[i]);
     consumer_sync();
