@@ -92,13 +92,16 @@ def measured_peaks() -> dict:
     return {}
 
 
-def profile_traffic(kernel_key: str, wl_name: str) -> float | None:
-    """DRAM bytes per launch from a committed ncu summary, if its kernel source is unchanged."""
+def profile_traffic(kernel_key: str, wl_name: str, summary_dtype: str = "fp32") -> float | None:
+    """DRAM bytes per launch from a committed ncu summary of the same kernel, workload and
+    summary storage type, if its kernel source is unchanged."""
     f = ROOT / "profiles" / f"{kernel_key}_{wl_name}.json"
     if not f.exists():
         return None
     try:
         rec = json.loads(f.read_text())
+        if rec.get("summary_dtype", "fp32") != summary_dtype:
+            return None
         if rec.get("source_sha256") != source_hash(rec.get("sources", [])):
             return None
         return float(rec["dram_bytes_per_launch"])
@@ -490,7 +493,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
                      "bytes_per_launch": nbytes["score_stream_kernel"], "us_per_launch": us_stream,
-                     "traffic": profile_traffic("score_stream_kernel", wl.name)},
+                     "traffic": profile_traffic("score_stream_kernel", wl.name, args.summary_dtype)},
         "kernels_us": {"score_stream": us_stream, "score_select": us_score,
                        "sparse_decode": us_sparse, "step": ms / args.steps * 1e3},
         "dense": {"ms_per_step": ms_dense, "steps_per_s": 1e3 / ms_dense,
