@@ -651,9 +651,6 @@ __device__ __forceinline__ int warp_sort_asc(int v) {
   return v;
 }
 
-// This CTA's 32 best codes of items [0, n) (code_at(i)), descending, in lists[0..31]. Each warp
-// scans a contiguous run in chunks of 32 (sort, merge into its running list); the 8 warp lists
-// then merge pairwise in 3 levels. `lists` needs kWarps * 32 entries. Contains CTA barriers.
 // Named CTA barriers over `n` threads (a multiple of 32): a producer arrives, a consumer waits.
 __device__ __forceinline__ void named_bar_arrive(int id, int n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -681,34 +678,6 @@ __device__ __forceinline__ uint64_t warp_pairs_merge_top32(uint64_t best, uint64
     id += kWarps / (2 * s);
   }
   return best;
-}
-
-// Merges the 8 warps' descending lists (`best` in each warp) into lists[0..31], pairwise in 3
-// levels. `lists` needs kWarps * 32 entries. Contains CTA barriers.
-__device__ __forceinline__ void cta_merge_warp_lists(uint64_t best, uint64_t* lists) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  lists[warp * 32 + lane] = best;
-  __syncthreads();
-#pragma unroll
-  for (int s = 1; s < kWarps; s <<= 1) {
-    if ((warp & (2 * s - 1)) == 0) best = warp_merge_top32(best, lists[(warp + s) * 32 + lane]);
-    __syncthreads();
-    if ((warp & (2 * s - 1)) == 0) lists[warp * 32 + lane] = best;
-    __syncthreads();
-  }
-}
-
-template <typename CodeAt>
-__device__ void cta_top32(CodeAt code_at, int n, uint64_t* lists) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int span = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-  const int i0 = warp * span, i1 = min(n, i0 + span);
-  uint64_t best = 0;
-  for (int b = i0; b < i1; b += 32) {
-    const int i = b + lane;
-    best = warp_merge_top32(best, warp_sort_desc(i < i1 ? code_at(i) : 0ull));
-  }
-  cta_merge_warp_lists(best, lists);
 }
 
 }  // namespace compkv
