@@ -40,6 +40,7 @@
 
 #include "attend.cuh"
 #include "common.cuh"
+#include "topk_lists.cuh"
 #include "internal.h"
 
 namespace cg = cooperative_groups;
@@ -48,7 +49,10 @@ namespace compkv {
 namespace {
 
 constexpr int kMaxCluster = 16;
-constexpr int kWarpTopK = 32;  // K_b up to this: warp bitonic Top-K; above: radix select
+constexpr int kWarpTopK = 128;  // K_b up to this: warp bitonic Top-K (lists of 32 LS); above: radix
+
+// Entries per lane of the warp Top-K lists for K_b (lists of 32, 64 or 128 codes).
+__host__ __device__ inline int list_slots(int Kb) { return Kb <= 32 ? 1 : (Kb <= 64 ? 2 : 4); }
 
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
@@ -63,7 +67,10 @@ struct FLay {
     ccap = Kb < chunk ? Kb : chunk;
     gcap = ccap * C;
     size_t o = 0;
-    hist = o;   o = a16(o + sizeof(uint32_t) * 2592);
+    // radix histograms, or the warp Top-K's lists: [kWarps] warp lists, [kMaxCluster] pushed
+    // rank lists and 2 x [kWarps] merge levels, of 32 * list_slots(K_b) codes each
+    const size_t lists = sizeof(uint64_t) * (3 * kWarps + kMaxCluster) * 32 * list_slots(Kb);
+    hist = o;   o = a16(o + (Kb <= kWarpTopK && lists > sizeof(uint32_t) * 2592 ? lists : sizeof(uint32_t) * 2592));
     keys = o;   o = a16(o + sizeof(uint32_t) * chunk);
     ck = o;     o = a16(o + sizeof(uint32_t) * (ccap + 1));
     ci = o;     o = a16(o + sizeof(int) * (ccap + 1));
@@ -173,7 +180,8 @@ __device__ __forceinline__ int stream_cta_of_tile(long long f, int nctas, int F)
 }
 
 
-template <typename T, int D, int G, typename S>  // S: summary storage type (float or __half)
+// S: summary storage type (float or __half); LS: entries per lane of the warp Top-K lists.
+template <typename T, int D, int G, typename S, int LS>
 __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_constant__ FParams p) {
   constexpr int XS = xrec_stride(G);
   extern __shared__ __align__(128) unsigned char sm[];
@@ -218,7 +226,8 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   //   mbar[1]  this rank's selection slots, from rank 0 (warp Top-K path)
   //   mbar[2]  merging ranks: the C partials of their output slice and (M, L) of its heads
   constexpr int E = G * D;
-  const bool warp_topk = p.do_select && p.Kb > 0 && p.Kb <= kWarpTopK;
+  const bool warp_topk = p.do_select && p.Kb > 0 && p.Kb <= 32 * LS;
+  constexpr int LW = 32 * LS;  // entries of a warp Top-K list
   const int first_owner = (p.do_select && C > 1) ? 1 : 0;
   const int n_owners = C - first_owner;
   const int per_o = (E + n_owners - 1) / n_owners;
@@ -231,7 +240,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     mbar_init(&mbar[1], 1);
     mbar_init(&mbar[2], 1);
     mbar_init_fence();
-    if (warp_topk && rank == 0) mbar_arrive_expect_tx(&mbar[0], static_cast<uint32_t>(C * 32 * 8));
+    if (warp_topk && rank == 0) mbar_arrive_expect_tx(&mbar[0], static_cast<uint32_t>(C * LW * 8));
     if (warp_topk && p.do_attend && my_slots > 0) mbar_arrive_expect_tx(&mbar[1], static_cast<uint32_t>(my_slots * 4));
     if (p.do_attend && oe0 < oe1) {
       const int nh = (oe1 - 1) / D - oe0 / D + 1;
@@ -322,26 +331,52 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       return empty ? 0u : score_key(S);
     };
     if (tid == 0) misc[0] = 0;
-    uint64_t best = 0ull;  // warp 0 ends with this rank's best-32 list (warp Top-K path)
+    uint64_t* h64 = reinterpret_cast<uint64_t*>(hist);
+    uint64_t best[LS];  // warp 0 ends with this rank's best-LW list (warp Top-K path)
+#pragma unroll
+    for (int e = 0; e < LS; ++e) best[e] = 0ull;
     if (warp_topk) {
-      // this rank's best 32 (descending codes) in hist[0..255]: a superset of its share. Chunks
-      // go in pairs: two independent sorts, then one merge.
-      best = 0ull;
-      for (int k = 0; k * 32 < span; k += 2) {
-        const int ja = jb + k * 32 + lane, jc = ja + 32;
-        const uint32_t ka = key_of(k, ja);
-        const uint32_t kc = ((k + 1) * 32 < span) ? key_of(k + 1, jc) : 0u;
-        const uint64_t sa = warp_sort_desc(ja < nloc ? topk_code(ka, j0 + ja) : 0ull);
-        const uint64_t sc = warp_sort_desc(((k + 1) * 32 < span && jc < nloc) ? topk_code(kc, j0 + jc) : 0ull);
-        const uint64_t m2 = warp_merge_top32(sa, sc);
-        best = (k == 0) ? m2 : warp_merge_top32(best, m2);
+      // this rank's best LW (descending codes): a superset of its share
+      if constexpr (LS == 1) {
+        // chunks go in pairs: two independent sorts, then one merge
+        for (int k = 0; k * 32 < span; k += 2) {
+          const int ja = jb + k * 32 + lane, jc = ja + 32;
+          const uint32_t ka = key_of(k, ja);
+          const uint32_t kc = ((k + 1) * 32 < span) ? key_of(k + 1, jc) : 0u;
+          const uint64_t sa = warp_sort_desc(ja < nloc ? topk_code(ka, j0 + ja) : 0ull);
+          const uint64_t sc = warp_sort_desc(((k + 1) * 32 < span && jc < nloc) ? topk_code(kc, j0 + jc) : 0ull);
+          const uint64_t m2 = warp_merge_top32(sa, sc);
+          best[0] = (k == 0) ? m2 : warp_merge_top32(best[0], m2);
+        }
+        best[0] = warp_pairs_merge_top32(best[0], h64);  // warp 0: the rank's list
+      } else {
+        // chunks of 32 go LS at a time: one list sort, then a merge into the running list
+        for (int c0 = 0; c0 * 32 < span; c0 += LS) {
+          uint64_t v[LS];
+#pragma unroll
+          for (int e = 0; e < LS; ++e) {
+            const int c = c0 + e, j = jb + c * 32 + lane;
+            v[e] = 0ull;
+            if (c * 32 < span) {
+              const uint32_t key = key_of(c, j);
+              if (j < nloc) v[e] = topk_code(key, j0 + j);
+            }
+          }
+          list_sort_desc<LS>(v);
+          if (c0 == 0) {
+#pragma unroll
+            for (int e = 0; e < LS; ++e) best[e] = v[e];
+          } else {
+            list_merge_top<LS>(best, v);
+          }
+        }
+        list_pairs_merge<LS>(best, h64);  // warp 0: the rank's list
       }
-      best = warp_pairs_merge_top32(best, reinterpret_cast<uint64_t*>(hist));  // warp 0: the rank's list
       if (p.do_attend && warp == 0) {
         // speculative: this rank's likeliest picks start moving from HBM to L2 while the global
         // cut runs (about 2 K_b / C of them: the global Top-K_b holds K_b / C per rank on average)
         const int m = min(32, max(1, (2 * Kb + C - 1) / C));
-        const uint64_t code = best;
+        const uint64_t code = best[0];
         if (lane < m && code != 0ull) {
           const int j = topk_index(code);
           const size_t off = (static_cast<size_t>(pr) * p.T + static_cast<size_t>(j) * kBlockTokens) * D;
@@ -378,33 +413,48 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     }
     cluster_wait();  // every rank has started: peers' shared memory may be written
     if (warp_topk && warp == 0) {  // push this rank's list into rank 0
-      const uint64_t code = best;
-      st_async_b64(cluster_smem_addr(reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + rank * 32 + lane, 0), code,
-                   cluster_smem_addr(&mbar[0], 0));
+#pragma unroll
+      for (int e = 0; e < LS; ++e)
+        st_async_b64(cluster_smem_addr(h64 + kWarps * LW + rank * LW + e * 32 + lane, 0), best[e],
+                     cluster_smem_addr(&mbar[0], 0));
     }
     if (!warp_topk) cluster.sync();  // #1 (radix path): every rank's candidates are visible
 
     // ---- 2. rank 0: global Top-K_b from the ranks' candidates; other ranks: compensation merge
-    if (rank == 0 && Kb > 0 && Kb <= kWarpTopK) {
-      // merge the C ranks' best-32 lists pairwise (the first level straight from the ranks'
+    if (rank == 0 && warp_topk) {
+      // merge the C ranks' best-LW lists pairwise (the first level straight from the ranks'
       // shared memory), then order the first K_b by block index
       mbar_wait_cluster(&mbar[0], 0, p.status);  // the C lists have arrived
-      const uint64_t* rl = reinterpret_cast<const uint64_t*>(hist) + kWarps * 32;  // [C][32] pushed
-      uint64_t* g0 = reinterpret_cast<uint64_t*>(hist) + kWarps * 32 + kMaxCluster * 32;
-      uint64_t* g1 = g0 + kWarps * 32;
+      const uint64_t* rl = h64 + kWarps * LW;    // [C][LW] pushed
+      uint64_t* g0 = h64 + kWarps * LW + kMaxCluster * LW;
+      uint64_t* g1 = g0 + kWarps * LW;
+      // list o of `from` and list o + 1, merged into list w of `to` (one warp)
+      auto merge_pair = [&](const uint64_t* from, int o, uint64_t* to, int w) {
+        uint64_t a[LS], b[LS];
+#pragma unroll
+        for (int e = 0; e < LS; ++e) {
+          a[e] = from[o * LW + e * 32 + lane];
+          b[e] = from[(o + 1) * LW + e * 32 + lane];
+        }
+        list_merge_top<LS>(a, b);
+#pragma unroll
+        for (int e = 0; e < LS; ++e) to[w * LW + e * 32 + lane] = a[e];
+      };
       int nl = 1;
       if (C == 1) {
-        if (warp == 0) g0[lane] = rl[lane];
+        if (warp == 0) {
+#pragma unroll
+          for (int e = 0; e < LS; ++e) g0[e * 32 + lane] = rl[e * 32 + lane];
+        }
       } else {
-        if (warp < C / 2) g0[warp * 32 + lane] = warp_merge_top32(rl[2 * warp * 32 + lane], rl[(2 * warp + 1) * 32 + lane]);
+        if (warp < C / 2) merge_pair(rl, 2 * warp, g0, warp);
         nl = C / 2;
       }
       __syncthreads();
       uint64_t* src = g0;
       uint64_t* dst = g1;
       while (nl > 1) {
-        if (warp < nl / 2)
-          dst[warp * 32 + lane] = warp_merge_top32(src[2 * warp * 32 + lane], src[(2 * warp + 1) * 32 + lane]);
+        if (warp < nl / 2) merge_pair(src, 2 * warp, dst, warp);
         __syncthreads();
         uint64_t* t = src;
         src = dst;
@@ -412,17 +462,39 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         nl /= 2;
       }
       if (warp == 0) {
-        const int idx = warp_sort_asc(lane < Kb ? topk_index(src[lane]) : 0x7fffffff);
-        if (lane < Kb && p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + lane] = idx;
-        if (p.do_attend) {
-          // lane r pushes rank r's slots [r per, r per + per) into its shared memory; rank r
-          // starts as soon as its bytes land, with no cluster barrier
-          for (int q = 0; q < per_slot; ++q) {
-            const int slot = lane * per_slot + q;
-            const int v = __shfl_sync(0xffffffffu, idx, slot < 32 ? slot : 0);
-            if (lane < C && slot < Kb)
-              st_async_b32(cluster_smem_addr(&selm[q], lane), static_cast<uint32_t>(v),
-                           cluster_smem_addr(&mbar[1], lane));
+        if constexpr (LS == 1) {
+          const int idx = warp_sort_asc(lane < Kb ? topk_index(src[lane]) : 0x7fffffff);
+          if (lane < Kb && p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + lane] = idx;
+          if (p.do_attend) {
+            // lane r pushes rank r's slots [r per, r per + per) into its shared memory; rank r
+            // starts as soon as its bytes land, with no cluster barrier
+            for (int q = 0; q < per_slot; ++q) {
+              const int slot = lane * per_slot + q;
+              const int v = __shfl_sync(0xffffffffu, idx, slot < 32 ? slot : 0);
+              if (lane < C && slot < Kb)
+                st_async_b32(cluster_smem_addr(&selm[q], lane), static_cast<uint32_t>(v),
+                             cluster_smem_addr(&mbar[1], lane));
+            }
+          }
+        } else {
+          int v[LS];
+#pragma unroll
+          for (int e = 0; e < LS; ++e) {
+            const int i = e * 32 + lane;
+            v[e] = i < Kb ? topk_index(src[i]) : 0x7fffffff;
+          }
+          list_sort_asc<LS>(v);
+#pragma unroll
+          for (int e = 0; e < LS; ++e) {
+            const int i = e * 32 + lane;  // the i-th selected block in block order
+            if (i < Kb) {
+              if (p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + i] = v[e];
+              if (p.do_attend) {  // slot i goes to rank i / per_slot, which starts when its bytes land
+                const int r = i / per_slot;
+                st_async_b32(cluster_smem_addr(&selm[i - r * per_slot], r), static_cast<uint32_t>(v[e]),
+                             cluster_smem_addr(&mbar[1], r));
+              }
+            }
           }
         }
         if (lane == 0) misc[6] = Kb;
@@ -768,27 +840,48 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   cluster_wait();  // no CTA leaves while a peer's push into it may be in flight
 }
 
-template <typename T, int D, typename S>
+template <typename T, int D, typename S, int LS>
 const void* kptr_g(int G) {
   switch (G) {
-    case 1: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 1, S>);
-    case 2: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 2, S>);
-    case 4: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 4, S>);
-    case 8: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 8, S>);
+    case 1: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 1, S, LS>);
+    case 2: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 2, S, LS>);
+    case 4: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 4, S, LS>);
+    case 8: return reinterpret_cast<const void*>(&decode_fused_kernel<T, D, 8, S, LS>);
   }
   return nullptr;
 }
 
+template <typename S, int LS>
+const void* pick_se(bool bf16, int D, int G) {
+  if (bf16) return D == 128 ? kptr_g<uint16_t, 128, S, LS>(G) : (D == 64 ? kptr_g<uint16_t, 64, S, LS>(G) : nullptr);
+  return D == 128 ? kptr_g<float, 128, S, LS>(G) : (D == 64 ? kptr_g<float, 64, S, LS>(G) : nullptr);
+}
 
 template <typename S>
-const void* pick_s(bool bf16, int D, int G) {
-  if (bf16) return D == 128 ? kptr_g<uint16_t, 128, S>(G) : (D == 64 ? kptr_g<uint16_t, 64, S>(G) : nullptr);
-  return D == 128 ? kptr_g<float, 128, S>(G) : (D == 64 ? kptr_g<float, 64, S>(G) : nullptr);
+const void* pick_s(bool bf16, int D, int G, int ls) {
+  switch (ls) {
+    case 2: return pick_se<S, 2>(bf16, D, G);
+    case 4: return pick_se<S, 4>(bf16, D, G);
+    default: return pick_se<S, 1>(bf16, D, G);
+  }
 }
 
-const void* pick(bool bf16, int D, int G, bool fp16) {
-  return fp16 ? pick_s<__half>(bf16, D, G) : pick_s<float>(bf16, D, G);
+// The kernel for `ls` entries per lane of the Top-K lists (1 also serves the radix path).
+const void* pick(bool bf16, int D, int G, bool fp16, int ls) {
+  return fp16 ? pick_s<__half>(bf16, D, G, ls) : pick_s<float>(bf16, D, G, ls);
 }
+
+// Preferred cluster size: the largest power of two <= 16 that keeps the grid within two CTAs
+// per SM and at least 64 blocks per rank.
+int preferred_cluster(int pairs, int Nb, int sms) {
+  int C0 = 1;
+  while (C0 < kMaxCluster && pairs * (2 * C0) <= 2 * sms && (Nb + 2 * C0 - 1) / (2 * C0) >= 64) C0 *= 2;
+  return C0;
+}
+
+// Lists above 32 entries pay a sort of every 32 of a rank's blocks per list entry slot; with
+// more than this many blocks per rank the radix cut is cheaper (measured at 4096 blocks).
+constexpr int kListMaxChunk = 1024;
 
 // Launch plan of one problem shape: the cluster size and the shared-memory layout.
 struct Plan {
@@ -825,8 +918,7 @@ cudaError_t make_plan(const void* kern, const FusedArgs& a, Plan* out) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  int C0 = 1;
-  while (C0 < kMaxCluster && a.pairs * (2 * C0) <= 2 * sms && (a.Nb + 2 * C0 - 1) / (2 * C0) >= 64) C0 *= 2;
+  const int C0 = preferred_cluster(a.pairs, a.Nb, sms);
   for (int C = C0; C >= 1; C /= 2) {
     const int chunk = (a.Nb + C - 1) / C;
     FLay L;
@@ -857,10 +949,13 @@ cudaError_t make_plan(const void* kern, const FusedArgs& a, Plan* out) {
 }  // namespace
 
 cudaError_t launch_decode_fused(const FusedArgs& a, cudaStream_t st) {
-  const void* kern = pick(a.bf16, a.D, a.G, a.fp16_summ);
-  if (!kern) return cudaErrorInvalidValue;
-  int dev = 0;
+  int dev = 0, sms = 0;
   cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int chunk0 = (a.Nb + preferred_cluster(a.pairs, a.Nb, sms) - 1) / preferred_cluster(a.pairs, a.Nb, sms);
+  const int ls = (a.Kb <= 32) ? 1 : ((a.Kb <= kWarpTopK && chunk0 <= kListMaxChunk) ? list_slots(a.Kb) : 1);
+  const void* kern = pick(a.bf16, a.D, a.G, a.fp16_summ, ls);
+  if (!kern) return cudaErrorInvalidValue;
   Plan plan;
   {
     std::lock_guard<std::mutex> lock(g_mu);
