@@ -87,13 +87,14 @@ def test_decode_head_layouts(G, d, dtype):
     P.check_step(run, 256, "compkv", all_pairs(wl))
 
 
-def test_decode_fused_equals_separate_calls():
+@pytest.mark.parametrize("budget", [512, 1024, 2048])   # Top-K lists of 32, 64 and 128 entries
+def test_decode_fused_equals_separate_calls(budget):
     wl = L32.with_(ctx_len=16384)
-    a = P.run_step(P.upload(wl), 512, "compkv", fused=True)
-    b = P.run_step(P.upload(wl), 512, "compkv", fused=False)
+    a = P.run_step(P.upload(wl), budget, "compkv", fused=True)
+    b = P.run_step(P.upload(wl), budget, "compkv", fused=False)
     assert torch.equal(a.sel, b.sel)
     assert torch.equal(a.out, b.out)
-    c = P.run_step(P.upload(wl), 512, "compkv", fused=True)
+    c = P.run_step(P.upload(wl), budget, "compkv", fused=True)
     assert torch.equal(a.out, c.out) and torch.equal(a.scores, c.scores)   # deterministic
 
 
