@@ -15,10 +15,11 @@
 //     candidates: its own best under (S desc, index asc).
 //  2. Rank 0 takes the global Top-K_b from the C candidate lists, read over distributed shared
 //     memory; the global Top-K_b under this strict order always lies inside the union of the
-//     local ones, so the result is exact. For K_b <= 32 the lists are each rank's best 32 as
-//     64-bit codes (key, then index), built and merged with warp bitonic networks; above that,
-//     radix selection. Meanwhile the other ranks merge the compensation partials of the
-//     kv-head's segments, a slice of channels each.
+//     local ones, so the result is exact. For K_b <= 32, and for K_b <= 128 when a rank holds
+//     at most 1024 blocks, the lists are each rank's best 32 LS as 64-bit codes (key, then
+//     index; LS = 1, 2 or 4 entries per lane), built and merged with warp bitonic networks;
+//     otherwise radix selection. Meanwhile the other ranks merge the compensation partials of
+//     the kv-head's segments, a slice of channels each.
 //  3. Rank c attends the c-th contiguous slice of rank 0's ordered selection (balanced whatever
 //     the blocks' positions; rank 0 writes each rank's slots into its shared memory and releases
 //     them through st.async bytes counted on the rank's mbarrier): their K and V rows read
