@@ -1,0 +1,59 @@
+"""Host-side pieces of bench.py that need no GPU: the algorithmic byte count of a step and the
+DRAM-traffic record read from a committed ncu summary (only for the same summary storage type
+and only while the kernel's sources are unchanged)."""
+import hashlib
+import json
+import pathlib
+
+import bench
+from sparse_kv_cache_summaries_b200 import synth
+
+
+def test_step_bytes_at_128k_512():
+    wl = synth.WORKLOADS["llama8b_128k_b512"]
+    fp32 = bench.step_bytes(wl, "fp32")
+    fp16 = bench.step_bytes(wl, "fp16")
+    # 8 kv-heads x 8192 blocks x (2 x 128 x 4 + 4 x (4 + 1)) bytes of summaries
+    assert fp32["summaries"] == 8 * 8192 * 1044
+    assert fp16["summaries"] == 8 * 8192 * (2 * 128 * 2 + 4 * 5)
+    # 32 selected blocks of 16 bf16 K and V rows per kv-head
+    assert fp32["selected_kv"] == fp16["selected_kv"] == 8 * 32 * 16 * 128 * 2 * 2
+    assert fp32["step"] == 70541312
+    assert fp32["score_stream_kernel"] == 68427776
+
+
+def _fake_root(tmp_path: pathlib.Path, summary_dtype: str | None) -> pathlib.Path:
+    src = tmp_path / "k.cu"
+    src.write_text("// kernel source\n")
+    rec = {"kernel": "score_stream_kernel", "workload": "w", "dram_bytes_per_launch": 123.0,
+           "sources": ["k.cu"], "source_sha256": hashlib.sha256(src.read_bytes()).hexdigest()}
+    if summary_dtype is not None:
+        rec["summary_dtype"] = summary_dtype
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "score_stream_kernel_w.json").write_text(json.dumps(rec))
+    return tmp_path
+
+
+def test_traffic_record_is_keyed_by_summary_dtype(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path, "fp32"))
+    assert bench.profile_traffic("score_stream_kernel", "w", "fp32") == 123.0
+    assert bench.profile_traffic("score_stream_kernel", "w", "fp16") is None
+    assert bench.profile_traffic("score_stream_kernel", "other", "fp32") is None
+
+
+def test_traffic_record_without_dtype_means_fp32(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", _fake_root(tmp_path, None))
+    assert bench.profile_traffic("score_stream_kernel", "w", "fp32") == 123.0
+    assert bench.profile_traffic("score_stream_kernel", "w", "fp16") is None
+
+
+def test_traffic_record_goes_stale_with_the_source(tmp_path, monkeypatch):
+    root = _fake_root(tmp_path, "fp32")
+    monkeypatch.setattr(bench, "ROOT", root)
+    (root / "k.cu").write_text("// kernel source, changed\n")
+    assert bench.profile_traffic("score_stream_kernel", "w", "fp32") is None
+
+
+def test_committed_traffic_record_matches_the_sources():
+    # the committed summary of the roofline kernel is current for the sources it names
+    assert bench.profile_traffic("score_stream_kernel", "llama8b_128k_b512", "fp32") is not None
