@@ -52,3 +52,13 @@ def test_traffic_record_goes_stale_with_the_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", root)
     (root / "k.cu").write_text("// kernel source, changed\n")
     assert bench.profile_traffic("score_stream_kernel", "w", "fp32") is None
+
+
+def test_clock_records_that_cannot_stand():
+    ok = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 30}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected({**ok, "sm_mhz": 1300, "reasons": ["sw_power_cap"]})
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected({**ok, "reasons": ["sw_power_cap", r]})
+    assert bench.clocks_rejected({**ok, "sm_mhz": 1000})            # a leftover clock lock
+    assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0})
