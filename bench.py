@@ -10,11 +10,16 @@ The default workload is the Llama-3.1-8B layer at 128K context with a 512-token 
 
 Timing: R = 4 independent caches (K, V, summaries) are resident in HBM and the steps rotate
 through them, so the per-step working set (about 70 MB at 128K) times R exceeds the 126 MB L2.
-Steps are replayed from CUDA graphs; the timed region is bracketed by a barrier and
-torch.cuda.synchronize, timed with CUDA events on the launching stream, and the max over ranks
-is taken. Several N run as independent replicas (weak scaling, no collective on the data path).
+Steps are replayed from CUDA graphs. After a warm-up of at least --warmup steps and at least
+WARMUP_S seconds, the timed region of exactly --steps steps is run many times (at least
+MIN_REGIONS, and enough to fill MIN_WINDOW_S seconds); each region is bracketed by a barrier and
+torch.cuda.synchronize and timed with CUDA events on the launching stream. The reported time per
+step is the median region divided by --steps, then the max over ranks. NVML samples the SM clock
+and the throttle reasons over the whole window of timed regions. Several N run as independent
+replicas (weak scaling, no collective on the data path).
 
-`--impl reference` times the fp64 CPU oracle on this host's cores instead (rank 0 only).
+`--impl reference` times the fp64 CPU oracle on this host's cores instead (rank 0 only): whole
+decode steps, BLAS threads = all cores, and it reports the number of steps it actually timed.
 """
 from __future__ import annotations
 
@@ -36,6 +41,13 @@ METRIC = "decode attn steps/s & HBM GB/s (% of peak) at 128K ctx, 512-tok budget
 UNIT = "steps/s"
 N_CACHES = 4
 FALLBACK_HBM_GBS = 6650.0
+WARMUP_S = 0.5        # seconds of graph replays before the first timed region
+MIN_REGIONS = 50      # timed regions of --steps steps, at least
+MIN_WINDOW_S = 0.5    # ... and enough regions to fill this many seconds (clock sampling)
+MAX_WINDOW_S = 20.0   # ... but no more than this many
+KERNELS_PER_STEP = 2  # this library's kernels launched per decode step
+STEP_GRAPH = ("CUDA graphs; streaming score kernel, then the select-and-attend kernel with "
+              "programmatic dependent launch")
 
 
 def parse():
@@ -48,7 +60,6 @@ def parse():
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--dense-steps", type=int, default=200)
     ap.add_argument("--summary-dtype", default="fp32", choices=["fp32", "fp16"],
                     help="storage of the mean key / mean value summaries")
     return ap.parse_args()
@@ -159,18 +170,19 @@ class ClockSampler:
             self.th.join(timeout=1)
 
     def summary(self, t0: float, t1: float) -> dict:
+        """Median SM clock and the union of throttle reasons over the samples in [t0, t1]."""
         win = [s for s in self.samples if t0 <= s[0] <= t1]
-        if len(win) < 3:   # the timed region was too short for the 20 ms sampler: widen it
-            win = [s for s in self.samples if t0 - 0.5 <= s[0] <= t1 + 0.1]
         if not win:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "sampler_ok": self.ok}
         reasons = set()
         for s in win:
             for name, bit in self.REASONS.items():
                 if s[2] & bit:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(win)}
+                "reasons": sorted(reasons), "samples": len(win), "sampler_ok": self.ok,
+                "window_s": t1 - t0}
 
 
 THROTTLE_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
@@ -207,18 +219,16 @@ def throughput(world: int, steps: int, ms_max: float) -> float:
 # ---------------------------------------------------------------------------------- reference
 
 def run_reference(args, rank: int):
-    """fp64 oracle on the host cores, on a bounded sample of the same workload."""
+    """The fp64 oracle, as it stands, on this host's cores: whole decode steps of the same
+    workload (summaries prebuilt), BLAS threads = all cores. It times `steps` steps, or as many
+    whole steps as fit in about two minutes, and reports the count it actually timed."""
     if rank != 0:
         return
-    import numpy as np
-    from threadpoolctl import threadpool_limits
-
-    import oracle
-    from sparse_kv_cache_summaries_b200 import synth
     wl = workload(args.workload, args.budget)
-    res = cpu_oracle_sample(wl, target_s=60.0, max_units=args.steps)
+    res = cpu_oracle_steps(wl, steps=max(1, args.steps), warmup=min(args.warmup, 2),
+                           threads=os.cpu_count() or 1, time_cap_s=120.0)
     line = {"impl": "reference", "metric": METRIC, "value": res["steps_per_s"], "unit": UNIT,
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "n_gpus": args.gpus, "steps": res["steps"], "warmup": res["warmup"],
             "ms_per_step": 1e3 / res["steps_per_s"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(wl),
@@ -227,39 +237,71 @@ def run_reference(args, rank: int):
             "e2e": {"value": res["steps_per_s"], "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-    del np, threadpool_limits, oracle, synth
 
 
-def cpu_oracle_sample(wl, target_s: float, max_units: int | None = None) -> dict:
-    """Times the oracle's decode step (summaries prebuilt) one (sequence, kv-head) at a time, in
-    order, until about `target_s` seconds of work; returns full steps per second."""
-    import numpy as np
-    from threadpoolctl import threadpool_limits
+def _oracle_unit(oracle, wl, q, K, V, summ, g):
+    """The oracle's decode step for one (sequence, kv-head): score, Top-K, compensated attention
+    of the kv-head's query heads (summaries prebuilt)."""
+    G = wl.group_size
+    s = oracle.default_scale(wl.head_dim)
+    S = oracle.group_scores(q[g * G:(g + 1) * G], summ[g], s)
+    sel = oracle.select_blocks(S, oracle.n_select(wl.budget, 16, S.shape[0]))
+    kg, vg = oracle.compkv._f64(K[g]), oracle.compkv._f64(V[g])
+    for h in range(G):
+        oracle.compensated_attention(q[g * G + h], kg, vg, summ[g], sel, s, 16)
 
+
+def _oracle_inputs(wl):
     import oracle
     from sparse_kv_cache_summaries_b200 import synth
     q, K, V = synth.make_sequence(wl, 0)
-    pairs = wl.batch * wl.n_kv_heads
-    G = wl.group_size
-    with threadpool_limits(limits=1):
-        summ = [oracle.block_summaries(K[g], V[g], 16, wl.n_groups) for g in range(wl.n_kv_heads)]
+    summ = [oracle.block_summaries(K[g], V[g], 16, wl.n_groups) for g in range(wl.n_kv_heads)]
+    return oracle, q, K, V, summ
+
+
+def cpu_oracle_steps(wl, steps: int, warmup: int, threads: int, time_cap_s: float) -> dict:
+    """Times whole decode steps of the oracle (every (sequence, kv-head) of sequence 0's layer,
+    batch 1 shape; for B > 1 a step repeats it B times), up to `steps` or until `time_cap_s`."""
+    from threadpoolctl import threadpool_limits
+    oracle, q, K, V, summ = _oracle_inputs(wl)
+    per_step = wl.batch * wl.n_kv_heads
+
+    def one_step():
+        for u in range(per_step):
+            _oracle_unit(oracle, wl, q, K, V, summ, u % wl.n_kv_heads)
+
+    with threadpool_limits(limits=threads):
+        for _ in range(warmup):
+            one_step()
         done, t_total = 0, 0.0
-        while t_total < target_s and (max_units is None or done < max_units):
-            g = done % wl.n_kv_heads
+        while done < steps and (done == 0 or t_total < time_cap_s):
             t0 = time.perf_counter()
-            S = oracle.group_scores(q[g * G:(g + 1) * G], summ[g], oracle.default_scale(wl.head_dim))
-            sel = oracle.select_blocks(S, oracle.n_select(wl.budget, 16, S.shape[0]))
-            kg, vg = oracle.compkv._f64(K[g]), oracle.compkv._f64(V[g])
-            for h in range(G):
-                oracle.compensated_attention(q[g * G + h], kg, vg, summ[g], sel,
-                                             oracle.default_scale(wl.head_dim), 16)
+            one_step()
+            t_total += time.perf_counter() - t0
+            done += 1
+    return {"steps_per_s": done / t_total, "steps": done, "warmup": warmup, "cores": threads,
+            "seconds": t_total,
+            "sample": f"{done} whole decode steps of {wl.name} ({per_step} (sequence, kv-head) "
+                      f"units each), summaries prebuilt, numpy fp64, BLAS threads = {threads}"}
+
+
+def cpu_oracle_sample(wl, target_s: float, threads: int = 1) -> dict:
+    """Times the oracle's decode step (summaries prebuilt) one (sequence, kv-head) at a time, in
+    order, until about `target_s` seconds of work; returns full steps per second."""
+    from threadpoolctl import threadpool_limits
+    oracle, q, K, V, summ = _oracle_inputs(wl)
+    pairs = wl.batch * wl.n_kv_heads
+    with threadpool_limits(limits=threads):
+        done, t_total = 0, 0.0
+        while t_total < target_s:
+            t0 = time.perf_counter()
+            _oracle_unit(oracle, wl, q, K, V, summ, done % wl.n_kv_heads)
             t_total += time.perf_counter() - t0
             done += 1
     steps = done / pairs
-    del np
-    return {"steps_per_s": steps / t_total, "cores": 1, "seconds": t_total,
+    return {"steps_per_s": steps / t_total, "cores": threads, "seconds": t_total,
             "sample": f"{done} (sequence, kv-head) units = {steps:.3f} decode steps of "
-                      f"{wl.name}, summaries prebuilt, numpy fp64, BLAS limited to 1 thread"}
+                      f"{wl.name}, summaries prebuilt, numpy fp64, BLAS threads = {threads}"}
 
 
 def config_of(wl, summary_dtype: str = "fp32") -> dict:
@@ -269,7 +311,100 @@ def config_of(wl, summary_dtype: str = "fp32") -> dict:
             "input_dtype": wl.dtype, "summary_dtype": summary_dtype,
             "l2": f"rotates {N_CACHES} independent caches; working set "
                   f"{N_CACHES} x step bytes > 126 MB L2",
-            "graph": "CUDA graphs; streaming score kernel, then the select-and-attend kernel with programmatic dependent launch"}
+            "graph": STEP_GRAPH}
+
+
+# ---------------------------------------------------------------------------------- timing
+
+def region_counts(est_region_ms: float, min_regions: int = MIN_REGIONS,
+                  min_window_s: float = MIN_WINDOW_S, max_window_s: float = MAX_WINDOW_S) -> int:
+    """How many timed regions to run: at least `min_regions`, and enough to fill `min_window_s`
+    (so the clock sampler sees the load), but no more than `max_window_s` worth."""
+    est = max(est_region_ms, 1e-3) / 1e3
+    n = max(min_regions, math.ceil(min_window_s / est))
+    cap = max(min_regions, int(max_window_s / est))
+    return min(n, cap)
+
+
+class GraphSet:
+    """CUDA graphs of a per-cache step function: one graph of `chunk` steps over the rotating
+    caches (replayed for long regions) and one graph per remainder length, so a region of n steps
+    is n graph steps with no host launch between them."""
+
+    def __init__(self, torch, stream, caches, fn, steps: int, chunk_cap: int = 256):
+        self.torch, self.stream = torch, stream
+        self.chunk = min(steps, chunk_cap)
+        self.chunk -= self.chunk % len(caches) if self.chunk >= len(caches) else 0
+        self.chunk = max(1, self.chunk)
+        self.graphs = {}
+        self._capture(caches, fn, self.chunk)
+        rem = steps % self.chunk
+        if rem:
+            self._capture(caches, fn, rem)
+
+    def _capture(self, caches, fn, n):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(self.stream):
+            with torch.cuda.graph(g, stream=self.stream):
+                for i in range(n):
+                    fn(caches[i % len(caches)])
+        self.graphs[n] = g
+
+    def replay(self, n: int):
+        full, rem = divmod(n, self.chunk)
+        for _ in range(full):
+            self.graphs[self.chunk].replay()
+        if rem:
+            self.graphs[rem].replay()
+
+
+def timed_regions(torch, stream, graphs: GraphSet, steps: int, world: int, device,
+                  warmup_steps: int = 0, warmup_s: float = 0.0, regions: int | None = None):
+    """Warm-up (at least `warmup_steps` steps and `warmup_s` seconds of replays), then `regions`
+    timed regions of exactly `steps` steps each, every region bracketed by a barrier and a
+    synchronize, timed with CUDA events on the launching stream. Every rank runs the same number
+    of regions (the max over ranks of each rank's own count). Returns (per-region ms list, wall
+    window (t0, t1))."""
+    t_end = time.perf_counter() + warmup_s
+    done = 0
+    with torch.cuda.stream(stream):
+        while done < warmup_steps or time.perf_counter() < t_end:
+            graphs.replay(steps if steps <= 4096 else 4096)
+            done += steps if steps <= 4096 else 4096
+            stream.synchronize()
+
+    def one():
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            graphs.replay(steps)
+            e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1)
+
+    if regions is None:
+        probe = one()
+        regions = region_counts(probe)
+        regions = int(max_over_ranks([float(regions)], device)[0])
+    t0 = time.perf_counter()
+    times = [one() for _ in range(regions)]
+    t1 = time.perf_counter()
+    if world > 1:
+        torch.distributed.barrier()
+    return times, (t0, t1)
+
+
+def region_stats(times_ms, steps: int) -> dict:
+    """Median (the reported figure), min and max of the per-region times, per step in µs."""
+    return {"regions": len(times_ms), "steps_per_region": steps,
+            "median_us_per_step": statistics.median(times_ms) / steps * 1e3,
+            "min_us_per_step": min(times_ms) / steps * 1e3,
+            "max_us_per_step": max(times_ms) / steps * 1e3}
 
 
 # ---------------------------------------------------------------------------------- ours
@@ -296,7 +431,6 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     stream = torch.cuda.Stream(device=dev)
 
     caches = []
-    build_times = []
     for i in range(N_CACHES):
         q, K, V = synth.make_batch(wl.with_(seed=wl.seed + 1000 * i + 97 * rank))
         c = {"q": q.to(dev), "K": K.to(dev), "V": V.to(dev)}
@@ -306,15 +440,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         c["ws"] = ck.new_workspace(shape, wl.budget, dev)
         c["dense_ws"] = ck.new_full_workspace(shape, dev)
         c["dense_out"] = torch.empty_like(c["out"])
-        torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ck.build_summaries(shape, c["K"], c["V"], c["summ"], stream=stream)   # warm
-            e0.record(stream)
             ck.build_summaries(shape, c["K"], c["V"], c["summ"], stream=stream)
-            e1.record(stream)
         stream.synchronize()
-        build_times.append(e0.elapsed_time(e1))
         caches.append(c)
         del q, K, V
 
@@ -335,98 +463,47 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     def dense(c):
         ck.full_decode(shape, c["q"], c["K"], c["V"], c["dense_out"], c["dense_ws"], stream=stream)
 
+    def build(c):
+        ck.build_summaries(shape, c["K"], c["V"], c["summ"], stream=stream)
+
     # warm every path once (plans, attributes), then capture graphs
     with torch.cuda.stream(stream):
         for c in caches:
             step(c)
             dense(c)
     stream.synchronize()
+    steps = max(1, args.steps)
+    g_step = GraphSet(torch, stream, caches, step, steps)
 
-    def capture(fn, reps):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(g, stream=stream):
-                for _ in range(reps):
-                    for c in caches:
-                        fn(c)
-        return g
-
-    UNROLL = 8
-    paths = (("step", step), ("stream", stream_only), ("score", score_only), ("sparse", sparse_only))
-    big = {name: capture(fn, UNROLL) for name, fn in paths}
-    single = {k: [] for k in big}
-    for name, fn in paths:
-        for c in caches:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(stream):
-                with torch.cuda.graph(g, stream=stream):
-                    fn(c)
-            single[name].append(g)
-    per_big = UNROLL * N_CACHES
-
-    def replay(name, n):
-        full, rem = divmod(n, per_big)
-        for _ in range(full):
-            big[name].replay()
-        for i in range(rem):
-            single[name][i % N_CACHES].replay()
-
-    def timed(name, n):
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            replay(name, n)
-            e1.record(stream)
-        stream.synchronize()
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        return e0.elapsed_time(e1)
-
-    # a run whose clock record is rejected (on any rank) is measured once more
+    # the headline: a run whose clock record is rejected (on any rank) is measured once more
     for attempt in range(2):
         sampler = ClockSampler(local_rank).start()
-        with torch.cuda.stream(stream):
-            replay("step", args.warmup)
-        stream.synchronize()
-        t_wall0 = time.perf_counter()
-        ms = timed("step", args.steps)
-        t_wall1 = time.perf_counter()
-        clocks = sampler.summary(t_wall0, t_wall1)
+        times, (tw0, tw1) = timed_regions(torch, stream, g_step, steps, world, dev,
+                                          warmup_steps=args.warmup, warmup_s=WARMUP_S)
+        clocks = sampler.summary(tw0, tw1)
+        sampler.stop()
         rejected = max_over_ranks([1.0 if clocks_rejected(clocks) else 0.0], dev)[0] > 0
         if not rejected or attempt == 1:
             break
-        sampler.stop()
     if attempt == 1:
         clocks["remeasured"] = "the first run's clock record was rejected"
-    # per-kernel durations (same rotation, separately timed) for the roofline
-    with torch.cuda.stream(stream):
-        replay("stream", max(3, args.warmup // 4))
-    ms_stream = timed("stream", args.steps)
-    ms_score = timed("score", args.steps)
-    ms_sparse = timed("sparse", args.steps)
-    sampler.stop()
+    if clocks.get("samples", 0) < 3 and clocks.get("sampler_ok"):
+        raise RuntimeError(f"clock sampler saw {clocks.get('samples')} samples in the timed window")
+    stats = region_stats(times, steps)
+    us_step = max_over_ranks([stats["median_us_per_step"]], dev)[0]
 
-    ms, ms_stream, ms_score, ms_sparse = max_over_ranks([ms, ms_stream, ms_score, ms_sparse], dev)
+    # per-kernel durations for the roofline and the breakdown: same rotation, graphs, regions
+    def per_step_us(fn, n, warm_s=0.2):
+        gs = GraphSet(torch, stream, caches, fn, n)
+        t, _ = timed_regions(torch, stream, gs, n, world, dev, warmup_steps=n, warmup_s=warm_s)
+        return max_over_ranks([region_stats(t, n)["median_us_per_step"]], dev)[0]
 
-    # dense baseline (same caches, same rotation, eager launches)
-    nd = max(4, args.dense_steps)
-    with torch.cuda.stream(stream):
-        for c in caches:
-            dense(c)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(nd):
-            dense(caches[i % N_CACHES])
-        e1.record(stream)
-    stream.synchronize()
-    ms_dense = e0.elapsed_time(e1) / nd
+    n_k = min(steps, 256)
+    us_stream = per_step_us(stream_only, n_k)
+    us_score = per_step_us(score_only, n_k)
+    us_sparse = per_step_us(sparse_only, n_k)
+    us_dense = per_step_us(dense, min(steps, 32))
+    us_build = per_step_us(build, 4, warm_s=0.05)
 
     # end to end through the public API: pinned host q in, fp32 out back, every step
     e2e = None
@@ -434,7 +511,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         q_host = [c["q"].cpu().pin_memory() for c in caches]
         out_host = torch.empty(caches[0]["out"].shape, dtype=torch.float32).pin_memory()
         q_dev = [torch.empty_like(c["q"]) for c in caches]
-        n_e2e = min(args.steps, 5000)
+        n_e2e = max(steps if steps <= 5000 else 5000, 1)
 
         def e2e_step(i):
             c = caches[i % N_CACHES]
@@ -444,44 +521,59 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                            c["ws"], stream=stream)
             out_host.copy_(c["out"], non_blocking=True)
 
+        def e2e_region(n):
+            torch.cuda.synchronize()
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for i in range(n):
+                    e2e_step(i)
+                e1.record(stream)
+            stream.synchronize()
+            return e0.elapsed_time(e1)
+
         with torch.cuda.stream(stream):
-            for i in range(min(50, args.warmup + 8)):
+            t_end = time.perf_counter() + 0.2
+            i = 0
+            while i < 50 or time.perf_counter() < t_end:
                 e2e_step(i)
+                i += 1
         stream.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(n_e2e):
-                e2e_step(i)
-            e1.record(stream)
-        stream.synchronize()
-        ms_e2e = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+        reg = region_counts(e2e_region(n_e2e), min_regions=5, min_window_s=0.3, max_window_s=5.0)
+        reg = int(max_over_ranks([float(reg)], dev)[0])
+        t_e2e = [e2e_region(n_e2e) for _ in range(reg)]
+        ms_e2e = max_over_ranks([statistics.median(t_e2e)], dev)[0]
         e2e = {"value": throughput(world, n_e2e, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
-               "steps": n_e2e, "path": "compkv_decode_step via the Python binding, eager launches"}
+               "steps": n_e2e, "regions": reg,
+               "path": "compkv_decode_step via the Python binding, eager launches; median region"}
 
-    # incremental append of one token per sequence (timed on a copy of one cache's summaries)
+    # incremental append of one token per sequence (on a copy of one cache's summaries): device
+    # time per call from a graph of appends, and the host-bound eager rate through the binding
     c0 = caches[0]
     sa = ck.Summaries(*(t.clone() for t in (c0["summ"].mean_k, c0["summ"].var_g,
                                             c0["summ"].mean_v, c0["summ"].count)))
     k_new = c0["K"][:, :, -1].contiguous()
     v_new = c0["V"][:, :, -1].contiguous()
     pos = torch.full((wl.batch,), wl.ctx_len - 1, dtype=torch.int32, device=dev)
+
+    def app(_c):
+        ck.append(shape, k_new, v_new, pos, sa, stream=stream)
+
+    append_us = per_step_us(app, 64, warm_s=0.05)
     n_app = 200
     with torch.cuda.stream(stream):
-        for _ in range(10):
-            ck.append(shape, k_new, v_new, pos, sa, stream=stream)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(n_app):
-            ck.append(shape, k_new, v_new, pos, sa, stream=stream)
+            app(None)
         e1.record(stream)
     stream.synchronize()
-    append_us = e0.elapsed_time(e1) / n_app * 1e3
+    append_eager_us = e0.elapsed_time(e1) / n_app * 1e3
     del sa
 
     status = max(ck.read_device_status(c["ws"], stream) for c in caches)
@@ -492,22 +584,22 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peaks = measured_peaks()
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-    sec_step = ms / 1e3 / args.steps
-    us_stream = ms_stream / args.steps * 1e3
-    us_score = ms_score / args.steps * 1e3
-    us_sparse = ms_sparse / args.steps * 1e3
-    gbs_step = nbytes["step"] / sec_step / 1e9
+    gbs_step = nbytes["step"] / (us_step * 1e-6) / 1e9
     achieved = nbytes["score_stream_kernel"] / (us_stream * 1e-6) / 1e9
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        res = cpu_oracle_sample(wl, target_s=12.0)
-        cpu = {"value": res["steps_per_s"], "unit": UNIT, "cores": res["cores"], "kind": "oracle",
-               "sample": res["sample"]}
+        allc = cpu_oracle_sample(wl, target_s=10.0, threads=os.cpu_count() or 1)
+        one = cpu_oracle_sample(wl, target_s=10.0, threads=1)
+        cpu = {"value": allc["steps_per_s"], "unit": UNIT, "cores": allc["cores"], "kind": "oracle",
+               "sample": allc["sample"],
+               "single_thread": {"value": one["steps_per_s"], "cores": 1, "sample": one["sample"]}}
     line = {
-        "metric": METRIC, "value": throughput(world, args.steps, ms), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "metric": METRIC, "value": throughput(world, steps, us_step * steps / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": us_step / 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": config_of(wl, args.summary_dtype),
+        "timing": {**stats, "reported": "median over the timed regions; max over ranks",
+                   "warmup_s": WARMUP_S},
         "hbm": {"gbs": gbs_step, "bytes_per_step": nbytes["step"], "peak_gbs": peak,
                 "frac_of_" + peak_src: gbs_step / peak, "frac_of_nominal_8000": gbs_step / 8000.0},
         "roofline": {"kernel": "score_stream_kernel (scores, records and compensation partials "
@@ -517,14 +609,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "bytes_per_launch": nbytes["score_stream_kernel"], "us_per_launch": us_stream,
                      "traffic": profile_traffic("score_stream_kernel", wl.name, args.summary_dtype)},
         "kernels_us": {"score_stream": us_stream, "score_select": us_score,
-                       "sparse_decode": us_sparse, "step": ms / args.steps * 1e3},
-        "dense": {"ms_per_step": ms_dense, "steps_per_s": 1e3 / ms_dense,
-                  "gbs": nbytes["dense"] / (ms_dense / 1e3) / 1e9,
-                  "frac_of_" + peak_src: nbytes["dense"] / (ms_dense / 1e3) / 1e9 / peak,
-                  "speedup_sparse_over_dense": ms_dense / (ms / args.steps)},
-        "build_summaries_ms": statistics.median(build_times),
-        "append_us": append_us,
-        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
+                       "sparse_decode": us_sparse, "step": us_step},
+        "dense": {"ms_per_step": us_dense / 1e3, "steps_per_s": 1e6 / us_dense,
+                  "gbs": nbytes["dense"] / (us_dense * 1e-6) / 1e9,
+                  "frac_of_" + peak_src: nbytes["dense"] / (us_dense * 1e-6) / 1e9 / peak,
+                  "speedup_sparse_over_dense": us_dense / us_step},
+        "build_summaries_ms": us_build / 1e3,
+        "append_us": append_us, "append_eager_us": append_eager_us,
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": KERNELS_PER_STEP * steps * stats["regions"],
         "clocks": clocks, "device_status": status,
     }
     print(json.dumps(line), flush=True)

@@ -239,18 +239,25 @@ int compkv_full_decode(const compkv_shape* shape, compkv_dtype dtype, const void
  *   - Shapes whose compkv_workspace_bytes(shape, budget_tokens) exceeds
  *     COMPKV_STATIC_SCRATCH_BYTES are rejected with COMPKV_ERR_WORKSPACE_TOO_SMALL before any
  *     launch (the 128K-context, 8-kv-head layer needs about 4 MB).
- *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current) and keeps it; make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, a host-side lookup once the library's device code is loaded; the
+ *     first call on a device may load it, so make that first call before any stream capture).
  *   - Every call shares the one array, which keeps the previous call's contents. Nothing in it has
- *     to start at zero (each call overwrites what it reads); its device status word is not
- *     reported by this entry point. Calls that can overlap on the GPU (other streams, other host
- *     threads) race on the array: the caller must serialise them.
+ *     to start at zero (each call overwrites what it reads). A kernel that gives up an internal
+ *     wait records it in the array's status word, which compkv_static_read_device_status reads
+ *     and clears. Calls that can overlap on the GPU (other streams, other host threads) race on
+ *     the array: the caller must serialise them.
  * Arguments and outputs are those of compkv_decode_step without workspace and workspace_bytes. */
 int compkv_decode_step_static(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
                               const void* q, const void* K, const void* V, const void* mean_k,
                               const float* var_g, const void* mean_v, const int32_t* count,
                               int32_t budget_tokens, float softmax_scale, int32_t* sel_idx,
                               float* scores, float* out, void* stream);
+
+/* compkv_read_device_status for the scratch array of compkv_decode_step_static on the current
+ * device: copies its status word (COMPKV_DEVERR_* bits, 0 = clean) to *status (host) and clears
+ * it. Synchronises `stream`; allocates nothing. */
+int compkv_static_read_device_status(void* stream, int32_t* status);
 
 /* ------------------------------------------------------------------------------------------ */
 /* Diagnostics                                                                                  */

@@ -96,6 +96,7 @@ def lib() -> ctypes.CDLL:
             "compkv_decode_step_static": (ctypes.c_int, [SP, ctypes.c_int, ctypes.c_int, P, P, P,
                                                          P, P, P, P, I32, F, P, P, P, P]),
             "compkv_read_device_status": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
+            "compkv_static_read_device_status": (ctypes.c_int, [P, ctypes.POINTER(I32)]),
             "compkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "compkv_last_cuda_error": (ctypes.c_char_p, []),
             "compkv_version": (ctypes.c_int, []),
@@ -282,4 +283,12 @@ def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     st = ctypes.c_int32(0)
     _ok(lib().compkv_read_device_status(_p(workspace), _stream(stream), ctypes.byref(st)),
         "read_device_status")
+    return st.value
+
+
+def static_read_device_status(stream=None) -> int:
+    """Status word of the scratch array that decode_step_static uses (read and cleared)."""
+    st = ctypes.c_int32(0)
+    _ok(lib().compkv_static_read_device_status(_stream(stream), ctypes.byref(st)),
+        "static_read_device_status")
     return st.value

@@ -2,7 +2,6 @@
 // caller workspace, for callers that can hand the library inputs and outputs but cannot allocate
 // device memory themselves.
 #include <cstdint>
-#include <mutex>
 
 #include "compkv.h"
 
@@ -12,25 +11,17 @@ static __device__ __align__(256) unsigned char g_compkv_static_scratch[COMPKV_ST
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
 // Device address of the scratch array on the current device. The host-side symbol is only a
-// stand-in for it, so the address is looked up once per device, with that device current.
+// stand-in for it, so the address is looked up with that device current, on every call: a
+// cached address would go stale if the context were torn down (cudaDeviceReset) and the module
+// loaded again, and the lookup is a host-side table read once the module is loaded.
 int scratch_for_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return COMPKV_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_compkv_static_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return COMPKV_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_compkv_static_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return COMPKV_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return COMPKV_OK;
 }
 
@@ -53,4 +44,12 @@ extern "C" int compkv_decode_step_static(const compkv_shape* shape, compkv_dtype
   return compkv_decode_step(shape, dtype, mode, q, K, V, mean_k, var_g, mean_v, count,
                             budget_tokens, softmax_scale, sel_idx, scores, out, ws,
                             static_cast<size_t>(COMPKV_STATIC_SCRATCH_BYTES), stream);
+}
+
+extern "C" int compkv_static_read_device_status(void* stream, int32_t* status) {
+  if (status == nullptr) return COMPKV_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  const int st = scratch_for_current_device(&ws);
+  if (st != COMPKV_OK) return st;
+  return compkv_read_device_status(ws, stream, status);
 }

@@ -380,6 +380,33 @@ def check_fp16_storage():
     assert np.array_equal(s.mean_k[2], mu.astype(np.float16).astype(np.float64))
 
 
+def _binary16_value(bits: int) -> float:
+    """The value of an IEEE 754 binary16 bit pattern, decoded by its definition."""
+    sign = -1.0 if bits >> 15 else 1.0
+    e, f = (bits >> 10) & 0x1F, bits & 0x3FF
+    if e == 0:
+        return sign * math.ldexp(f, -24)          # subnormal: 2^-14 x f / 1024
+    assert e != 0x1F, "no inf / NaN in these cases"
+    return sign * math.ldexp(1024 + f, e - 25)    # 2^(e-15) x (1 + f / 1024)
+
+
+def check_fp16_golden():
+    """fp16 storage against hand-derived binary16 patterns (golden file): ties to even, just
+    above a tie, the sign, an inexact decimal, the spacing of large values, the largest finite
+    value and the subnormals."""
+    g = json.loads((GOLDEN / "fp16_storage.json").read_text())
+    for case in g["cases"]:
+        m = ev(case["mean"])
+        want = _binary16_value(int(case["bits"], 16))
+        k = np.full((16, 2), m)
+        k[:, 1] = -m
+        v = np.full((16, 2), m)
+        h = O.block_summaries(k, v, 16, 1, storage="fp16")
+        assert h.mean_k[0, 0] == want and h.mean_k[0, 1] == -want, (case, h.mean_k[0], want)
+        assert h.mean_v[0, 0] == want, (case, h.mean_v[0], want)
+        assert h.count[0] == 16
+
+
 def check_fidelity_statistics():
     """Spearman and residual capture: closed forms and textbook cases (App. B.2 statistics)."""
     x = np.array([3.0, 1.0, 4.0, 1.5, 9.0, 2.6])
@@ -408,4 +435,4 @@ ALL_CHECKS = [check_summaries_library, check_summaries_identical_keys, check_app
               check_second_form_and_dense_limit, check_zero_residual_block, check_ties_and_order,
               check_second_order_limit, check_bruteforce_residual_topk,
               check_mass_only_reduction, check_gqa_normalisation, check_fidelity_statistics,
-              check_fp16_storage]
+              check_fp16_storage, check_fp16_golden]

@@ -1,6 +1,6 @@
 """Helpers for the GPU-vs-oracle parity tests.
 
-Tolerances (the bar the method's target sets; see the design doc for the derivation):
+Tolerances (the bar the method's target sets: bf16 inputs with fp32 accumulation):
 * summaries: max|gpu - ref| / max|ref| <= 1e-3 per tensor and (b, kv-head); counts exact;
 * selection: the selected block set equals the oracle's Top-K_b, except blocks whose oracle
   score lies within 1e-5 (relative) of the K_b-th largest score (near-ties, logged);

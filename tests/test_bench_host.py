@@ -62,3 +62,22 @@ def test_clock_records_that_cannot_stand():
         assert bench.clocks_rejected({**ok, "reasons": ["sw_power_cap", r]})
     assert bench.clocks_rejected({**ok, "sm_mhz": 1000})            # a leftover clock lock
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0})
+
+
+def test_region_counts_fill_the_clock_window():
+    # 20 steps of ~30 us: a 0.6 ms region; at least 50 regions and at least 0.5 s of them
+    n = bench.region_counts(0.6)
+    assert n >= bench.MIN_REGIONS and n * 0.6e-3 >= bench.MIN_WINDOW_S
+    # a long region: the minimum count, capped by the window's upper bound
+    assert bench.region_counts(1000.0) == bench.MIN_REGIONS
+    assert bench.region_counts(1000.0, min_regions=5, max_window_s=2.0) == 5
+
+
+def test_reference_arm_reports_the_steps_it_timed(capsys):
+    class A:
+        workload, budget, steps, warmup, gpus = "tiny", None, 3, 1, 1
+    bench.run_reference(A, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 3
+    assert line["cpu_baseline"]["cores"] >= 1
+    assert line["value"] == line["cpu_baseline"]["value"] == line["e2e"]["value"]

@@ -4,7 +4,9 @@ Sizes: the tiny case and shrunken Llama-layer caches that still span many 32-blo
 cluster ranks and a ragged tail run on every (b, kv-head); the full-size workloads (32K and 128K
 context, the 3 x 3 length/budget grid, the 16 x 64K batch) run in the launch configuration the
 benchmark times (decode_step: the streaming score kernel, then the select-and-attend kernel with
-programmatic dependent launch) and are checked on sampled (b, kv-head) pairs the oracle computes one by one.
+programmatic dependent launch) and are checked on every kv-head of the Llama layer (the batched
+workload: one kv-head of every sequence, all 8 kv-head indices covered), each pair computed by the
+oracle one by one.
 """
 import numpy as np
 import pytest
@@ -166,7 +168,7 @@ def _full(wl, pairs, budget=None, dense=False):
     run = P.upload(wl)
     budget = wl.budget if budget is None else budget
     P.run_step(run, budget, "compkv")
-    P.check_summaries(run, pairs[:2])
+    P.check_summaries(run, pairs)
     info = P.check_step(run, budget, "compkv", pairs)
     if dense:
         out = torch.empty_like(run.out)
@@ -181,7 +183,7 @@ def test_full_llama_32k():
 
 
 def test_full_llama_128k():
-    _full(L128, [(0, 0), (0, 3), (0, 7)], dense=True)
+    _full(L128, all_pairs(L128), dense=True)
 
 
 @pytest.mark.parametrize("ctx", [32768, 65536, 131072])
@@ -191,8 +193,8 @@ def test_full_grid(ctx):
     P.run_summaries(run)
     for budget in (512, 1024, 2048):
         P.run_step(run, budget, "compkv")
-        P.check_step(run, budget, "compkv", [(0, 1), (0, 6)])
+        P.check_step(run, budget, "compkv", all_pairs(wl))
 
 
 def test_full_batched_16x64k():
-    _full(BATCH, [(0, 0), (7, 3), (15, 7)])
+    _full(BATCH, [(b, (3 * b) % BATCH.n_kv_heads) for b in range(BATCH.batch)])

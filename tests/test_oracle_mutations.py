@@ -16,7 +16,7 @@ _orig = {name: getattr(O, name) for name in (
     "block_summaries", "logit_variance_estimate", "second_order_log_mass", "head_scores",
     "compensated_attention", "select_blocks", "block_mean_logits", "dense_attention",
     "group_scores", "token_logits", "block_residuals", "log_partitions", "append_token", "rank_correlation",
-    "residual_capture")}
+    "residual_capture", "store")}
 
 
 def _summaries_sample_var(k, v, block_size=16, n_groups=4):
@@ -149,7 +149,27 @@ def _capture_unnormalised(score, resid, k_sel):
     return float(resid[O.select_blocks(score, k_sel)].sum())
 
 
+def _store_fp16_toward_zero(x, storage):
+    """fp16 storage that truncates (rounds toward zero) instead of rounding to nearest even."""
+    if storage != "fp16":
+        return _orig["store"](x, storage)
+    x = np.asarray(x, dtype=np.float64)
+    h = x.astype(np.float16)
+    over = np.abs(h.astype(np.float64)) > np.abs(x)
+    h = np.where(over, np.nextafter(h, np.float16(0)), h)
+    return h.astype(np.float64)
+
+
+def _store_fp16_as_fp32(x, storage):
+    """fp16 storage that keeps fp32 precision (the rounding step applied at the wrong width)."""
+    if storage != "fp16":
+        return _orig["store"](x, storage)
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
 MUTATIONS = {
+    "fp16_storage_toward_zero": ("store", _store_fp16_toward_zero),
+    "fp16_storage_at_fp32": ("store", _store_fp16_as_fp32),
     "spearman_on_values": ("rank_correlation", _spearman_on_values),
     "capture_unnormalised": ("residual_capture", _capture_unnormalised),
     "append_squared_new_mean": ("append_token", _append_squared_new_mean),

@@ -36,6 +36,7 @@ def test_static_scratch_step_matches_workspace_step():
         ck.decode_step_static(s, run.qd, run.Kd, run.Vd, run.summ, wl.budget, sel, out)
         torch.cuda.synchronize()
         assert torch.equal(sel, ref_sel)
+        assert ck.static_read_device_status() == 0
         err = (out - ref_out).abs()
         assert bool((err <= P.OUT_ATOL + P.OUT_RTOL * ref_out.abs()).all()), float(err.max())
 
