@@ -45,9 +45,9 @@ WARMUP_S = 0.5        # seconds of graph replays before the first timed region
 MIN_REGIONS = 50      # timed regions of --steps steps, at least
 MIN_WINDOW_S = 0.5    # ... and enough regions to fill this many seconds (clock sampling)
 MAX_WINDOW_S = 20.0   # ... but no more than this many
-KERNELS_PER_STEP = 1  # this library's kernels launched per decode step
-STEP_GRAPH = ("CUDA graphs; one clustered decode-step kernel per step (score, Top-K and "
-              "compensated attention), programmatic dependent launch between steps")
+KERNELS_PER_STEP = 2  # this library's kernels launched per decode step
+STEP_GRAPH = ("CUDA graphs; streaming score kernel, then the select-and-attend kernel with "
+              "programmatic dependent launch")
 
 
 def parse():
@@ -90,7 +90,7 @@ def step_bytes(wl, summary_dtype: str = "fp32") -> dict:
     q = wl.batch * wl.n_q_heads * d * esz
     out = wl.batch * wl.n_q_heads * d * 4
     return {"step": summ + sel_kv + q + out, "summaries": summ, "selected_kv": sel_kv,
-            "stream_only": summ + q, "dense": pairs * wl.ctx_len * d * esz * 2 + q + out}
+            "score_stream_kernel": summ + q, "dense": pairs * wl.ctx_len * d * esz * 2 + q + out}
 
 
 def measured_peaks() -> dict:
@@ -429,7 +429,6 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                           summary_dtype=args.summary_dtype)
     kb = ck.num_selected(shape, wl.budget)
     stream = torch.cuda.Stream(device=dev)
-    launch_cfg = ck.step_launch_config(shape, wl.budget)
 
     caches = []
     for i in range(N_CACHES):
@@ -586,7 +585,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
     gbs_step = nbytes["step"] / (us_step * 1e-6) / 1e9
-    achieved = gbs_step  # the step is one launch of decode_step_kernel
+    achieved = nbytes["score_stream_kernel"] / (us_stream * 1e-6) / 1e9
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         allc = cpu_oracle_sample(wl, target_s=10.0, threads=os.cpu_count() or 1)
@@ -603,16 +602,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "warmup_s": WARMUP_S},
         "hbm": {"gbs": gbs_step, "bytes_per_step": nbytes["step"], "peak_gbs": peak,
                 "frac_of_" + peak_src: gbs_step / peak, "frac_of_nominal_8000": gbs_step / 8000.0},
-        "roofline": {"kernel": "decode_step_kernel (the whole step: every block's summaries, "
-                               "the selected blocks' K/V, q in, outputs out)",
+        "roofline": {"kernel": "score_stream_kernel (scores, records and compensation partials "
+                               "over every block's summaries)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
-                     "bytes_per_launch": nbytes["step"], "us_per_launch": us_step,
-                     "traffic": profile_traffic("decode_step_kernel", wl.name, args.summary_dtype)},
-        "kernels_us": {"step": us_step, "stream_only": us_stream,
-                       "stream_only_gbs": nbytes["stream_only"] / (us_stream * 1e-6) / 1e9,
-                       "score_select": us_score, "sparse_decode": us_sparse},
-        "launch": launch_cfg,
+                     "bytes_per_launch": nbytes["score_stream_kernel"], "us_per_launch": us_stream,
+                     "traffic": profile_traffic("score_stream_kernel", wl.name, args.summary_dtype)},
+        "kernels_us": {"score_stream": us_stream, "score_select": us_score,
+                       "sparse_decode": us_sparse, "step": us_step},
         "dense": {"ms_per_step": us_dense / 1e3, "steps_per_s": 1e6 / us_dense,
                   "gbs": nbytes["dense"] / (us_dense * 1e-6) / 1e9,
                   "frac_of_" + peak_src: nbytes["dense"] / (us_dense * 1e-6) / 1e9 / peak,

@@ -96,11 +96,9 @@ int32_t compkv_num_selected(const compkv_shape* shape, int32_t budget_tokens);
 
 /* Bytes of device workspace that compkv_score_select / compkv_sparse_decode / compkv_decode_step
  * need for this shape and budget. 0 on an invalid shape. The workspace carries, between
- * compkv_score_select and compkv_sparse_decode on one stream, every block's per-head record
- * x = s q_h . mu_j + log n_j and the Mean-compensation partial sums of the ranks that split each
- * (sequence, kv-head); the per-block log scores live there too when a rank's share does not fit
- * in shared memory. Its first 4 bytes are the device status word (compkv_read_device_status): zero
- * it once before first use (e.g. cudaMemsetAsync); nothing else in it needs initialising. */
+ * compkv_score_select and compkv_sparse_decode on one stream, the Mean-compensation partial sums
+ * over all blocks, the split partials and the merge counters. It must be zero-filled once before
+ * its first use (e.g. cudaMemsetAsync); the library keeps the counters at zero between calls. */
 size_t compkv_workspace_bytes(const compkv_shape* shape, int32_t budget_tokens);
 
 /* Bytes of device workspace for compkv_full_decode (same zero-fill rule). */
@@ -174,12 +172,12 @@ int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
                         float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
                         size_t workspace_bytes, void* stream);
 
-/* a1, the streaming part alone: the pass of compkv_score_select over every block's summaries
- * (mean keys, grouped variances and counts, then mean values in the compensating modes), with
- * the per-block scores, the rank partials of Zhat and of the compensation sum kept on chip, but
- * without the exchange between ranks, the selection or any output. Exposed so that the part of
- * the step that reads all the summaries (its bandwidth-bound part) can be timed on its own;
- * nothing is written. Arguments as for compkv_score_select.                                    */
+/* a1, first pass alone: the streaming pass of compkv_score_select over every block's summaries,
+ * without the selection. It leaves in the workspace each block's per-head log score and mean
+ * logit record and the per-segment partials of Zhat and of the compensation sum; nothing else is
+ * written. Exposed so that the pass that reads all the summaries (the bandwidth-bound part of the
+ * step) can be timed on its own; a following compkv_score_select recomputes everything it needs.
+ * Arguments as for compkv_score_select.                                                       */
 int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
                         const void* q, const void* mean_k, const float* var_g,
                         const void* mean_v, const int32_t* count, int32_t budget_tokens,
@@ -206,13 +204,9 @@ int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_m
                          size_t workspace_bytes, void* stream);
 
 /* One whole decode step: the result of compkv_score_select followed by compkv_sparse_decode, in
- * one kernel launch. A thread-block cluster of up to 16 CTAs (one per SM) splits each (sequence,
- * kv-head): every rank streams its share of the summaries, the ranks exchange their partials of
- * Zhat and their candidate lists through distributed shared memory, every rank derives the same
- * Top-K_b, attends its slice of it while the mean values still stream in, and the ranks merge
- * their partials of the outputs. The selection is also written to sel_idx (and S_j to scores
- * when given). Launched with programmatic dependent launch. The results are bitwise those of
- * compkv_score_select followed by compkv_sparse_decode. Arguments as above. */
+ * two kernels: the streaming score pass, then one kernel that selects and attends (launched with
+ * programmatic dependent launch so its prologue overlaps the first's tail; the selection is kept
+ * on chip and also written to sel_idx). Arguments as above. */
 int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
                        const void* q, const void* K, const void* V, const void* mean_k,
                        const float* var_g, const void* mean_v, const int32_t* count,
@@ -271,13 +265,6 @@ int compkv_static_read_device_status(void* stream, int32_t* status);
 /* Copies the workspace status word (COMPKV_DEVERR_* bits, 0 = clean) to *status (host) and
  * clears it. Synchronises `stream`. */
 int compkv_read_device_status(void* workspace, void* stream, int32_t* status);
-
-/* Launch configuration the decode-step kernel uses for this shape and budget on the current
- * device (host pointers, any may be NULL): the ranks per (sequence, kv-head) cluster, the blocks
- * each rank owns, and the dynamic shared memory per CTA. Returns a negative status for an invalid
- * shape or budget; no launch. */
-int compkv_step_launch_config(const compkv_shape* shape, int32_t budget_tokens,
-                              int32_t* cluster_ranks, int32_t* blocks_per_rank, size_t* smem_bytes);
 
 /* Static, NUL-terminated description of a compkv_status value. */
 const char* compkv_status_string(int status);

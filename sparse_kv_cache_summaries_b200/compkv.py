@@ -97,9 +97,6 @@ def lib() -> ctypes.CDLL:
                                                          P, P, P, P, I32, F, P, P, P, P]),
             "compkv_read_device_status": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
             "compkv_static_read_device_status": (ctypes.c_int, [P, ctypes.POINTER(I32)]),
-            "compkv_step_launch_config": (ctypes.c_int, [SP, I32, ctypes.POINTER(I32),
-                                                         ctypes.POINTER(I32),
-                                                         ctypes.POINTER(SZ)]),
             "compkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "compkv_last_cuda_error": (ctypes.c_char_p, []),
             "compkv_version": (ctypes.c_int, []),
@@ -153,15 +150,6 @@ def num_selected(shape: LayerShape, budget_tokens: int) -> int:
     k = lib().compkv_num_selected(ctypes.byref(shape.c()), budget_tokens)
     _ok(min(k, 0), "num_selected")
     return k
-
-
-def step_launch_config(shape: LayerShape, budget_tokens: int) -> dict:
-    """Ranks per (sequence, kv-head) cluster, blocks per rank and shared memory per CTA of the
-    decode-step kernel on the current device."""
-    c, ch, sz = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_size_t(0)
-    _ok(lib().compkv_step_launch_config(ctypes.byref(shape.c()), budget_tokens, ctypes.byref(c),
-                                        ctypes.byref(ch), ctypes.byref(sz)), "step_launch_config")
-    return {"cluster_ranks": c.value, "blocks_per_rank": ch.value, "smem_bytes": sz.value}
 
 
 def workspace_bytes(shape: LayerShape, budget_tokens: int) -> int:

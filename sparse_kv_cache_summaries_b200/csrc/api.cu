@@ -183,55 +183,84 @@ int compkv_append(const compkv_shape* shape, compkv_dtype dtype, const void* k_n
   return cuda_status(compkv::launch_append(a, static_cast<cudaStream_t>(stream)));
 }
 
-// One launch of the decode-step kernel with the parts `sel`, `att`, `strm` (see StepArgs).
-static int step_impl(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
-                     const void* q, const void* K, const void* V, const void* mean_k,
-                     const float* var_g, const void* mean_v, const int32_t* count,
-                     int32_t budget_tokens, float softmax_scale, int32_t* sel_idx, float* scores,
-                     float* out, void* workspace, size_t workspace_bytes, void* stream, bool sel,
-                     bool att, bool strm) {
+enum class Upto { kStream, kSelect, kAttend };
+
+// Streaming score kernel, then (unless `upto` is kStream) the select kernel, or with kAttend the
+// select-and-attend kernel, launched with programmatic dependent launch.
+static int score_select_impl(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
+                             const void* q, const void* mean_k, const float* var_g,
+                             const void* mean_v, const int32_t* count, int32_t budget_tokens,
+                             float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
+                             size_t workspace_bytes, void* stream, Upto upto, const void* K,
+                             const void* V, float* out) {
   Common c;
   int st = check_step_args(shape, dtype, mode, budget_tokens, workspace, workspace_bytes, &c);
   if (st) return st;
   const bool comp = mode != COMPKV_MODE_MASS;
-  if (!q || (strm && (!mean_k || !var_g || !count)) || (strm && comp && !mean_v) ||
-      (att && (!K || !V || !out || !count || (comp && !mean_v))) || ((sel || att) && c.Kb > 0 && !sel_idx))
+  if (!q || !mean_k || !var_g || !count || (comp && !mean_v) ||
+      (upto != Upto::kStream && c.Kb > 0 && !sel_idx))
     return COMPKV_ERR_INVALID_ARG;
-  if (!aligned16(q) || (mean_k && !aligned16(mean_k)) || (mean_v && !aligned16(mean_v)) ||
-      (var_g && !aligned4(var_g)) || (count && !aligned4(count)) || (sel_idx && !aligned4(sel_idx)) ||
-      (scores && !aligned4(scores)) || (K && !aligned16(K)) || (V && !aligned16(V)) || (out && !aligned4(out)))
+  if (!aligned16(q) || !aligned16(mean_k) || (comp && !aligned16(mean_v)) || !aligned4(var_g) ||
+      !aligned4(count) || (sel_idx && !aligned4(sel_idx)) || (scores && !aligned4(scores)))
     return COMPKV_ERR_BAD_ALIGNMENT;
   const compkv::StepWorkspace W = step_ws(shape);
-  compkv::StepArgs a;
-  a.s.bf16 = dtype == COMPKV_BF16;
-  a.s.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
-  a.s.pairs = shape->batch * shape->n_kv_heads;
-  a.s.G = c.G;
-  a.s.D = shape->head_dim;
-  a.s.T = shape->ctx_len;
-  a.s.Nb = c.Nb;
-  a.s.Kb = c.Kb;
-  a.s.r = shape->n_groups;
+  const int pairs = shape->batch * shape->n_kv_heads;
+  int nctas = 0;
+  compkv::StreamArgs a;
+  a.bf16 = dtype == COMPKV_BF16;
+  a.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
   a.mode = mode;
-  a.do_select = sel;
-  a.do_attend = att;
-  a.do_stream = strm;
+  a.pairs = pairs;
+  a.G = c.G;
+  a.D = shape->head_dim;
+  a.Nb = c.Nb;
+  a.r = shape->n_groups;
+  a.slots = W.slots;
   a.scale = scale_of(shape, softmax_scale);
   a.q = q;
-  a.K = K;
-  a.V = V;
   a.mean_k = mean_k;
   a.var_g = var_g;
   a.mean_v = mean_v;
   a.count = count;
-  a.ug = ws_at(workspace, W.ug);
+  a.u = ws_at(workspace, W.u);
   a.xrec = ws_at(workspace, W.xrec);
-  a.cpart = ws_at(workspace, W.cpart);
-  a.sel_idx = sel_idx;
-  a.scores = scores;
-  a.out = out;
+  a.zpart = ws_at(workspace, W.zpart);
+  a.comp_seg = ws_at(workspace, W.comp_seg);
   a.status = status_word(workspace);
-  return cuda_status(compkv::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
+  a.nctas_out = &nctas;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int rc = cuda_status(compkv::launch_score_stream(a, cs));
+  if (rc || upto == Upto::kStream) return rc;
+  compkv::FusedArgs b;
+  b.bf16 = a.bf16;
+  b.fp16_summ = a.fp16_summ;
+  b.mode = mode;
+  b.do_select = true;
+  b.do_attend = upto == Upto::kAttend;
+  b.pairs = pairs;
+  b.G = c.G;
+  b.D = shape->head_dim;
+  b.T = shape->ctx_len;
+  b.Nb = c.Nb;
+  b.Kb = c.Kb;
+  b.slots = W.slots;
+  b.nctas_stream = nctas;
+  b.scale = a.scale;
+  b.q = q;
+  b.K = K;
+  b.V = V;
+  b.mean_v = mean_v;
+  b.u = a.u;
+  b.xrec = a.xrec;
+  b.zpart = a.zpart;
+  b.comp_seg = a.comp_seg;
+  b.comp = ws_at(workspace, W.comp);
+  b.sel_idx = sel_idx;
+  b.scores = scores;
+  b.out = out;
+  b.status = a.status;
+  b.pdl = true;
+  return cuda_status(compkv::launch_decode_fused(b, cs));
 }
 
 int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
@@ -239,9 +268,9 @@ int compkv_score_select(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
                         const void* mean_v, const int32_t* count, int32_t budget_tokens,
                         float softmax_scale, int32_t* sel_idx, float* scores, void* workspace,
                         size_t workspace_bytes, void* stream) {
-  return step_impl(shape, dtype, mode, q, nullptr, nullptr, mean_k, var_g, mean_v, count,
-                   budget_tokens, softmax_scale, sel_idx, scores, nullptr, workspace,
-                   workspace_bytes, stream, true, false, true);
+  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
+                           softmax_scale, sel_idx, scores, workspace, workspace_bytes, stream,
+                           Upto::kSelect, nullptr, nullptr, nullptr);
 }
 
 int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
@@ -249,9 +278,9 @@ int compkv_score_stream(const compkv_shape* shape, compkv_dtype dtype, compkv_mo
                         const void* mean_v, const int32_t* count, int32_t budget_tokens,
                         float softmax_scale, void* workspace, size_t workspace_bytes,
                         void* stream) {
-  return step_impl(shape, dtype, mode, q, nullptr, nullptr, mean_k, var_g, mean_v, count,
-                   budget_tokens, softmax_scale, nullptr, nullptr, nullptr, workspace,
-                   workspace_bytes, stream, false, false, true);
+  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
+                           softmax_scale, nullptr, nullptr, workspace, workspace_bytes, stream,
+                           Upto::kStream, nullptr, nullptr, nullptr);
 }
 
 int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
@@ -259,10 +288,46 @@ int compkv_sparse_decode(const compkv_shape* shape, compkv_dtype dtype, compkv_m
                          const void* mean_v, const int32_t* count, const int32_t* sel_idx,
                          int32_t budget_tokens, float softmax_scale, float* out, void* workspace,
                          size_t workspace_bytes, void* stream) {
-  // the selection is only read
-  return step_impl(shape, dtype, mode, q, K, V, mean_k, nullptr, mean_v, count, budget_tokens,
-                   softmax_scale, const_cast<int32_t*>(sel_idx), nullptr, out, workspace,
-                   workspace_bytes, stream, false, true, false);
+  Common c;
+  int st = check_step_args(shape, dtype, mode, budget_tokens, workspace, workspace_bytes, &c);
+  if (st) return st;
+  const bool comp = mode != COMPKV_MODE_MASS;
+  if (!q || !K || !V || !count || !out || (comp && (!mean_k || !mean_v)) || (c.Kb > 0 && !sel_idx))
+    return COMPKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || (comp && (!aligned16(mean_k) || !aligned16(mean_v))) ||
+      !aligned4(count) || (sel_idx && !aligned4(sel_idx)) || !aligned4(out))
+    return COMPKV_ERR_BAD_ALIGNMENT;
+  const compkv::StepWorkspace W = step_ws(shape);
+  compkv::FusedArgs b;
+  b.bf16 = dtype == COMPKV_BF16;
+  b.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
+  b.mode = mode;
+  b.do_select = false;
+  b.do_attend = true;
+  b.pairs = shape->batch * shape->n_kv_heads;
+  b.G = c.G;
+  b.D = shape->head_dim;
+  b.T = shape->ctx_len;
+  b.Nb = c.Nb;
+  b.Kb = c.Kb;
+  b.slots = W.slots;
+  b.nctas_stream = 0;
+  b.scale = scale_of(shape, softmax_scale);
+  b.q = q;
+  b.K = K;
+  b.V = V;
+  b.mean_v = mean_v;
+  b.u = nullptr;
+  b.xrec = ws_at(workspace, W.xrec);
+  b.zpart = nullptr;
+  b.comp_seg = nullptr;
+  b.comp = ws_at(workspace, W.comp);
+  b.sel_idx = const_cast<int32_t*>(sel_idx);  // read only when do_select is false
+  b.scores = nullptr;
+  b.out = out;
+  b.status = status_word(workspace);
+  b.pdl = false;
+  return cuda_status(compkv::launch_decode_fused(b, static_cast<cudaStream_t>(stream)));
 }
 
 int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mode mode,
@@ -272,9 +337,10 @@ int compkv_decode_step(const compkv_shape* shape, compkv_dtype dtype, compkv_mod
                        float* scores, float* out, void* workspace, size_t workspace_bytes,
                        void* stream) {
   if (!K || !V || !out) return COMPKV_ERR_INVALID_ARG;
-  return step_impl(shape, dtype, mode, q, K, V, mean_k, var_g, mean_v, count, budget_tokens,
-                   softmax_scale, sel_idx, scores, out, workspace, workspace_bytes, stream, true,
-                   true, true);
+  if (!aligned16(K) || !aligned16(V) || !aligned4(out)) return COMPKV_ERR_BAD_ALIGNMENT;
+  return score_select_impl(shape, dtype, mode, q, mean_k, var_g, mean_v, count, budget_tokens,
+                           softmax_scale, sel_idx, scores, workspace, workspace_bytes, stream,
+                           Upto::kAttend, K, V, out);
 }
 
 int compkv_full_decode(const compkv_shape* shape, compkv_dtype dtype, const void* q,
@@ -317,31 +383,6 @@ int compkv_read_device_status(void* workspace, void* stream, int32_t* status) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(int32_t), s);
   return cuda_status(e);
-}
-
-int compkv_step_launch_config(const compkv_shape* shape, int32_t budget_tokens,
-                              int32_t* cluster_ranks, int32_t* blocks_per_rank, size_t* smem_bytes) {
-  const int st = check_shape(shape);
-  if (st) return st;
-  if (budget_tokens < 0) return COMPKV_ERR_INVALID_ARG;
-  compkv::StepShape a;
-  a.bf16 = true;
-  a.fp16_summ = shape->summary_dtype == COMPKV_SUMMARY_FP16;
-  a.pairs = shape->batch * shape->n_kv_heads;
-  a.G = shape->n_q_heads / shape->n_kv_heads;
-  a.D = shape->head_dim;
-  a.T = shape->ctx_len;
-  a.Nb = n_blocks(shape);
-  a.Kb = kb_of(shape, budget_tokens);
-  a.r = shape->n_groups;
-  int C = 0, chunk = 0;
-  size_t smem = 0;
-  const int rc = cuda_status(compkv::step_plan(a, &C, &chunk, &smem));
-  if (rc) return rc;
-  if (cluster_ranks) *cluster_ranks = C;
-  if (blocks_per_rank) *blocks_per_rank = chunk;
-  if (smem_bytes) *smem_bytes = smem;
-  return COMPKV_OK;
 }
 
 const char* compkv_status_string(int status) {

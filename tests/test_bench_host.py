@@ -19,7 +19,7 @@ def test_step_bytes_at_128k_512():
     # 32 selected blocks of 16 bf16 K and V rows per kv-head
     assert fp32["selected_kv"] == fp16["selected_kv"] == 8 * 32 * 16 * 128 * 2 * 2
     assert fp32["step"] == 70541312
-    assert fp32["stream_only"] == 68427776
+    assert fp32["score_stream_kernel"] == 68427776
 
 
 def _fake_root(tmp_path: pathlib.Path, summary_dtype: str | None) -> pathlib.Path:
