@@ -2,12 +2,16 @@
 // measured against (CompKV review, Key claims and FAQ: speedup over full attention, Table 4).
 //
 // Split-K flash decode: the tokens of each (sequence, kv-head) are cut into `nsplit` contiguous
-// ranges, one CTA each, sized so the grid covers the SMs about three times. A CTA streams its
-// range in 32-token tiles of K and V through a 3-stage ring of bulk copies tracked by mbarriers,
-// computes the logits of the G query heads of the kv-head (transpose-reduced dot products),
-// updates an online softmax per head and accumulates P.V. Split partials (max, sum, acc) go to
-// the workspace; the last CTA of a kv-head to finish (atomic ticket, no waiting) merges them and
-// resets the ticket to zero for the next call.
+// ranges, one CTA each, about two CTAs per SM. A producer warp streams the range in 32-token
+// tiles of K and V (bulk copies into a ring of shared-memory stages with a "full" and an "empty"
+// mbarrier each); eight consumer warps each take 4 rows of every tile (2 rows at a time for 8
+// query heads per kv-head) and keep their own online softmax per query head, so no CTA barrier
+// is needed until the end: logits of the rows against the G query heads of the kv-head (each lane
+// holds D / 32 channels of a row; one transpose-reduce gives every lane one (row, head) logit),
+// the running max and sum, and P.V into per-lane accumulators. The 8 warps' partials merge in
+// shared memory into the split's partial (max, sum, acc) in the workspace; the last CTA of a
+// kv-head to finish (atomic ticket, no waiting) merges the splits and resets the ticket to zero
+// for the next call.
 #include "attend.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -15,11 +19,13 @@
 namespace compkv {
 namespace {
 
-constexpr int kTT = 32;      // tokens per tile
-constexpr int kStages = 3;
+constexpr int kTT = 32;                      // tokens per tile
+constexpr int kCons = 8;                     // consumer warps
+constexpr int kFThreads = (kCons + 1) * 32;  // + the producer warp
+constexpr int kMaxStages = 8;
 
 struct FParams {
-  int Hkv, T, nsplit;
+  int Hkv, T, nsplit, stages;
   float scale;
   const void* q;
   const void* K;
@@ -33,39 +39,47 @@ struct FParams {
 
 template <typename T, int D, int G>
 struct FLayout {
-  static constexpr size_t tile_bytes = sizeof(T) * kTT * D;
-  static constexpr size_t off_k = 0;                                        // [S][kTT][D]
-  static constexpr size_t off_v = off_k + kStages * tile_bytes;             // [S][kTT][D]
-  static constexpr size_t off_lg = off_v + kStages * tile_bytes;            // [G][kTT]
-  static constexpr size_t off_p = off_lg + sizeof(float) * G * kTT;         // [kTT][G]
-  static constexpr size_t off_q = off_p + sizeof(float) * G * kTT;          // [G][D]
-  static constexpr size_t off_red = off_q + sizeof(float) * G * D;          // [kSub][G][D]
-  static constexpr size_t off_ml = off_red + sizeof(float) * PV<T, D, G>::kSub * G * D;
-  static constexpr size_t off_sc = off_ml + sizeof(float) * 2 * 8;
-  static constexpr size_t off_flag = off_sc + sizeof(float) * 8;
-  static constexpr size_t off_mbar = (off_flag + 16 + 15) & ~size_t(15);
-  static constexpr size_t total = off_mbar + 8 * kStages;
+  static constexpr size_t tile_bytes = sizeof(T) * kTT * D;           // K (or V) rows of a tile
+  static constexpr size_t stage_bytes = 2 * tile_bytes;               // K, then V
+  static constexpr size_t off_q = 0;                                  // [G][D] fp32
+  static constexpr size_t off_wacc = off_q + sizeof(float) * G * D;   // [kCons][G][D]
+  static constexpr size_t off_wml = off_wacc + sizeof(float) * kCons * G * D;  // [kCons][G][2]
+  static constexpr size_t off_fac = off_wml + sizeof(float) * kCons * G * 2;   // [kCons][G], [G][2]
+  static constexpr size_t off_flag = off_fac + sizeof(float) * (kCons * G + 2 * G);
+  static constexpr size_t off_bar = (off_flag + 16 + 15) & ~size_t(15);        // full, empty
+  static constexpr size_t off_ring = (off_bar + 8 * 2 * kMaxStages + 127) & ~size_t(127);
+  static size_t total(int stages) { return off_ring + stage_bytes * stages; }
 };
 
+template <int G>
+__device__ __forceinline__ float pick_head(const float (&a)[G], int h) {
+  float v = a[0];
+#pragma unroll
+  for (int i = 1; i < G; ++i) v = (h == i) ? a[i] : v;
+  return v;
+}
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) full_decode_kernel(const __grid_constant__ FParams p) {
+__global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_constant__ FParams p) {
   using LY = FLayout<T, D, G>;
-  using RG = RowGeom<T, D>;
-  using PVt = PV<T, D, G>;
-  constexpr int EPV = RG::kEpv, VEC = PVt::kVec;
+  constexpr int VEP = D / 32;                // channels per lane
+  constexpr int GR = (G >= 8) ? 2 : 4;       // rows per group
+  constexpr int NV = GR * G;                 // (row, head) logits of a group
+  constexpr int LPV = 32 / NV;               // lanes per (row, head) after the reduce
+  constexpr int RPW = kTT / kCons;           // rows of a tile per consumer warp: 4
+  static_assert(NV <= 32 && RPW % GR == 0, "unsupported head layout");
   extern __shared__ __align__(128) unsigned char sm[];
-  T* kt = reinterpret_cast<T*>(sm + LY::off_k);
-  T* vt = reinterpret_cast<T*>(sm + LY::off_v);
-  float* lg = reinterpret_cast<float*>(sm + LY::off_lg);
-  float* pT = reinterpret_cast<float*>(sm + LY::off_p);
   float* q_s = reinterpret_cast<float*>(sm + LY::off_q);
-  float* red = reinterpret_cast<float*>(sm + LY::off_red);
-  float* ml_s = reinterpret_cast<float*>(sm + LY::off_ml);
-  float* sc_s = reinterpret_cast<float*>(sm + LY::off_sc);
+  float* wacc = reinterpret_cast<float*>(sm + LY::off_wacc);
+  float* wml = reinterpret_cast<float*>(sm + LY::off_wml);
+  float* fac = reinterpret_cast<float*>(sm + LY::off_fac);
   int* flag = reinterpret_cast<int*>(sm + LY::off_flag);
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + LY::off_mbar);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + LY::off_bar);
+  uint64_t* empty = full + kMaxStages;
+  unsigned char* ring = sm + LY::off_ring;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int NS = p.stages;
   const int bk = blockIdx.x / p.nsplit, split = blockIdx.x % p.nsplit;
   const int b = bk / p.Hkv;
   int Tb = p.ctx_lens ? p.ctx_lens[b] : p.T;
@@ -75,103 +89,208 @@ __global__ void __launch_bounds__(kThreads) full_decode_kernel(const __grid_cons
   const int ntiles = (t1 - t0 + kTT - 1) / kTT;
   const T* Kb = static_cast<const T*>(p.K) + (static_cast<size_t>(bk) * p.T + t0) * D;
   const T* Vb = static_cast<const T*>(p.V) + (static_cast<size_t>(bk) * p.T + t0) * D;
-  const uint64_t policy = l2_evict_first_policy();
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCons);
+    }
+    flag[1] = 0;
     mbar_init_fence();
   }
   {
     const T* qp = static_cast<const T*>(p.q) + static_cast<size_t>(bk) * G * D;
-    for (int i = tid; i < G * D; i += kThreads) q_s[i] = to_float(qp[i]);
+    for (int i = tid; i < G * D; i += kFThreads) q_s[i] = to_float(qp[i]);
   }
   __syncthreads();
-  auto issue = [&](int i) {
-    const int st = i % kStages;
-    const int rows = min(kTT, t1 - t0 - i * kTT);
-    const uint32_t bytes = static_cast<uint32_t>(rows) * D * sizeof(T);
-    mbar_arrive_expect_tx(&mbar[st], 2 * bytes);
-    bulk_g2s_stream(kt + static_cast<size_t>(st) * kTT * D, Kb + static_cast<size_t>(i) * kTT * D, bytes, &mbar[st], policy);
-    bulk_g2s_stream(vt + static_cast<size_t>(st) * kTT * D, Vb + static_cast<size_t>(i) * kTT * D, bytes, &mbar[st], policy);
-  };
-  if (tid == 0)
-    for (int i = 0; i < min(ntiles, kStages - 1); ++i) issue(i);
-  int issued = min(ntiles, kStages - 1), waited = ntiles;
 
-  const int li = lane % RG::kLpr;
-  float qr[G][EPV];
-  load_q_regs<T, D, G>(q_s, li, qr);
-  const int cv = tid % PVt::kCols, sub = tid / PVt::kCols;
-  float acc[G][VEC];
+  if (warp == kCons) {  // ---- producer: tile i into stage i % NS once its last use is released
+    const uint64_t policy = l2_evict_first_policy();
+    int issued = 0;
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % NS;
+      if (i >= NS) {
+        bool got = mbar_wait(&empty[st], static_cast<uint32_t>((i / NS - 1) & 1), p.status);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+          if (lane == 0) flag[1] = 1;
+          break;
+        }
+        fence_proxy_async();
+      }
+      if (lane == 0) {
+        const int rows = min(kTT, t1 - t0 - i * kTT);
+        const uint32_t bytes = static_cast<uint32_t>(rows) * D * sizeof(T);
+        unsigned char* sb = ring + LY::stage_bytes * st;
+        mbar_arrive_expect_tx(&full[st], 2 * bytes);
+        bulk_g2s_stream(sb, Kb + static_cast<size_t>(i) * kTT * D, bytes, &full[st], policy);
+        bulk_g2s_stream(sb + LY::tile_bytes, Vb + static_cast<size_t>(i) * kTT * D, bytes, &full[st], policy);
+      }
+      ++issued;
+    }
+    if (*reinterpret_cast<volatile int*>(&flag[1]) != 0) {  // gave up: drain the copies in flight
+      for (int i = max(0, issued - NS); i < issued; ++i)
+        mbar_wait(&full[i % NS], static_cast<uint32_t>((i / NS) & 1), nullptr);
+    }
+  } else {  // ---- consumers
+    float qv[G][VEP];
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[h][e] = 0.f;
-  float m_run = -CUDART_INF_F, l_run = 0.f;
-  bool ok = true;
-
-#pragma unroll 1
-  for (int i = 0; i < ntiles; ++i) {
-    const int st = i % kStages;
-    const int rows = min(kTT, t1 - t0 - i * kTT);
-    T* ks = kt + static_cast<size_t>(st) * kTT * D;
-    T* vs = vt + static_cast<size_t>(st) * kTT * D;
-    const bool got = mbar_wait(&mbar[st], (i / kStages) & 1, p.status);
-    if (rows < kTT) {  // ragged last tile: zero the V rows no copy wrote (their weight is 0)
-      for (int e = tid; e < (kTT - rows) * D; e += kThreads) vs[static_cast<size_t>(rows) * D + e] = T(0);
-    }
-    tile_logits<T, D, G>(ks, kTT, qr, p.scale, lg, kTT, [&](int row) { return row < rows; });
-    ok = __syncthreads_and(got) != 0;
-    if (!ok) {
-      waited = i;
-      break;
-    }
-    if (tid == 0 && i + kStages - 1 < ntiles) issue(i + kStages - 1);
-    if (i + kStages - 1 < ntiles) ++issued;
-    if (warp < G) {
-      const int h = warp;
-      const float x = lg[h * kTT + lane];
-      const float m_new = fmaxf(m_run, warp_max(x));
-      const float w = (x == -CUDART_INF_F) ? 0.f : __expf(x - m_new);
-      pT[lane * G + h] = w;
-      const float sc = (m_run == -CUDART_INF_F) ? 0.f : __expf(m_run - m_new);
-      l_run = l_run * sc + warp_sum(w);
-      m_run = m_new;
-      if (lane == 0) sc_s[h] = sc;
-    }
-    __syncthreads();
+      for (int e = 0; e < VEP; ++e) qv[h][e] = q_s[h * D + lane * VEP + e];
+    float acc[G][VEP], mw[G], lw[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float sc = sc_s[h];
+      mw[h] = -CUDART_INF_F;
+      lw[h] = 0.f;
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[h][e] *= sc;
+      for (int e = 0; e < VEP; ++e) acc[h][e] = 0.f;
     }
-    PVt::accumulate(vs, pT, kTT, sub, cv, acc);
-  }
-  if (!ok) {
-    for (int i = waited; i < issued; ++i) mbar_wait(&mbar[i % kStages], (i / kStages) & 1, nullptr);
+    const int my_v = lane / LPV, my_r = my_v / G, my_h = my_v % G;
+    bool ok = true;
+#pragma unroll 1
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % NS;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[st], static_cast<uint32_t>((i / NS) & 1), p.status));
+      const int rows = ok ? min(kTT, t1 - t0 - i * kTT) : 0;
+      const T* kt = reinterpret_cast<const T*>(ring + LY::stage_bytes * st);
+      const T* vt = reinterpret_cast<const T*>(ring + LY::stage_bytes * st + LY::tile_bytes);
+#pragma unroll
+      for (int g0 = 0; g0 < RPW; g0 += GR) {
+        const int r0 = warp * RPW + g0;  // the group's first row in the tile
+        if (r0 >= rows) break;
+        float v[NV];
+#pragma unroll
+        for (int r = 0; r < GR; ++r) {
+          float kf[VEP];
+          if (r0 + r < rows) {
+            const T* row = kt + (r0 + r) * D;
+            if constexpr (sizeof(T) == 2) {
+              if constexpr (VEP == 4) {
+                const uint2 w = reinterpret_cast<const uint2*>(row)[lane];
+                kf[0] = __uint_as_float(w.x << 16);
+                kf[1] = __uint_as_float(w.x & 0xffff0000u);
+                kf[2] = __uint_as_float(w.y << 16);
+                kf[3] = __uint_as_float(w.y & 0xffff0000u);
+              } else {
+                const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
+                kf[0] = __uint_as_float(w << 16);
+                kf[1] = __uint_as_float(w & 0xffff0000u);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < VEP; ++e) kf[e] = row[lane * VEP + e];
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < VEP; ++e) kf[e] = 0.f;
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEP; ++e) s = fmaf(qv[h][e], kf[e], s);
+            v[r * G + h] = s;
+          }
+        }
+        TransposeReduce<NV, 16>::run(v, lane);  // lane holds (row my_r, head my_h)
+        const float lg = (r0 + my_r < rows) ? p.scale * v[0] : -CUDART_INF_F;
+        float gm = lg;
+#pragma unroll
+        for (int o = LPV * G; o < 32; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+        float mn[G], sc[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float gh = __shfl_sync(0xffffffffu, gm, h * LPV);
+          mn[h] = fmaxf(mw[h], gh);
+          sc[h] = (mw[h] == -CUDART_INF_F) ? 0.f : __expf(mw[h] - mn[h]);
+        }
+        const float pe = (lg == -CUDART_INF_F) ? 0.f : __expf(lg - pick_head<G>(mn, my_h));
+        float ps = pe;
+#pragma unroll
+        for (int o = LPV * G; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          lw[h] = lw[h] * sc[h] + __shfl_sync(0xffffffffu, ps, h * LPV);
+          mw[h] = mn[h];
+#pragma unroll
+          for (int e = 0; e < VEP; ++e) acc[h][e] *= sc[h];
+        }
+#pragma unroll
+        for (int r = 0; r < GR; ++r) {
+          if (r0 + r < rows) {  // rows past the range carry weight 0 and are skipped
+            float vf[VEP];
+            const T* row = vt + (r0 + r) * D;
+            if constexpr (sizeof(T) == 2) {
+              if constexpr (VEP == 4) {
+                const uint2 w = reinterpret_cast<const uint2*>(row)[lane];
+                vf[0] = __uint_as_float(w.x << 16);
+                vf[1] = __uint_as_float(w.x & 0xffff0000u);
+                vf[2] = __uint_as_float(w.y << 16);
+                vf[3] = __uint_as_float(w.y & 0xffff0000u);
+              } else {
+                const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
+                vf[0] = __uint_as_float(w << 16);
+                vf[1] = __uint_as_float(w & 0xffff0000u);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < VEP; ++e) vf[e] = row[lane * VEP + e];
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float prh = __shfl_sync(0xffffffffu, pe, (r * G + h) * LPV);
+#pragma unroll
+              for (int e = 0; e < VEP; ++e) acc[h][e] = fmaf(prh, vf[e], acc[h][e]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    // this warp's partial
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < VEP; ++e) wacc[(warp * G + h) * D + lane * VEP + e] = acc[h][e];
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        wml[(warp * G + h) * 2] = mw[h];
+        wml[(warp * G + h) * 2 + 1] = lw[h];
+      }
+    }
   }
   __syncthreads();
 
-  // ---- split partial -> workspace
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) red[(sub * G + h) * D + cv * VEC + e] = acc[h][e];
-  if (warp < G && lane == 0) {
-    ml_s[2 * warp] = m_run;
-    ml_s[2 * warp + 1] = l_run;
+  // ---- the 8 warps' partials -> this split's partial in the workspace
+  float* mine = p.part + (static_cast<size_t>(bk) * p.nsplit + split) * G * (D + 2);
+  float* wf = fac;                 // [kCons][G] factors
+  float* sml = fac + kCons * G;    // [G][2] the split's (max, sum)
+  if (warp < G) {
+    const int h = warp;
+    const float mwv = lane < kCons ? wml[(lane * G + h) * 2] : -CUDART_INF_F;
+    const float M = warp_max(mwv);
+    const float f = exp_diff(mwv, M);
+    const float Ls = warp_sum(lane < kCons ? f * wml[(lane * G + h) * 2 + 1] : 0.f);
+    if (lane < kCons) wf[lane * G + h] = f;
+    if (lane == 0) {
+      sml[2 * h] = M;
+      sml[2 * h + 1] = Ls;
+    }
   }
   __syncthreads();
-  float* mine = p.part + (static_cast<size_t>(bk) * p.nsplit + split) * G * (D + 2);
-  for (int i = tid; i < G * D; i += kThreads) {
-    float s = 0.f;
-    for (int k = 0; k < PVt::kSub; ++k) s += red[k * G * D + i];
-    mine[(i / D) * (D + 2) + 2 + (i % D)] = s;
+  for (int i = tid; i < G * D; i += kFThreads) {
+    const int h = i / D;
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCons; ++w) a = fmaf(wf[w * G + h], wacc[(w * G + h) * D + (i % D)], a);
+    mine[h * (D + 2) + 2 + (i % D)] = a;
   }
   if (tid < G) {
-    mine[tid * (D + 2)] = ml_s[2 * tid];
-    mine[tid * (D + 2) + 1] = ml_s[2 * tid + 1];
+    mine[tid * (D + 2)] = sml[2 * tid];
+    mine[tid * (D + 2) + 1] = sml[2 * tid + 1];
   }
   __threadfence();
   __syncthreads();
@@ -182,6 +301,7 @@ __global__ void __launch_bounds__(kThreads) full_decode_kernel(const __grid_cons
   // ---- last CTA of this kv-head: merge the splits
   __threadfence();
   const float* parts = p.part + static_cast<size_t>(bk) * p.nsplit * G * (D + 2);
+  float* ml_s = sml;
   if (tid < G) {
     float M = -CUDART_INF_F;
     for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, __ldcg(parts + (static_cast<size_t>(s) * G + tid) * (D + 2)));
@@ -196,7 +316,7 @@ __global__ void __launch_bounds__(kThreads) full_decode_kernel(const __grid_cons
   }
   __syncthreads();
   float* o = p.out + static_cast<size_t>(bk) * G * D;
-  for (int i = tid; i < G * D; i += kThreads) {
+  for (int i = tid; i < G * D; i += kFThreads) {
     const int h = i / D, c = i % D;
     const float M = ml_s[2 * h];
     float a = 0.f;
@@ -210,10 +330,20 @@ __global__ void __launch_bounds__(kThreads) full_decode_kernel(const __grid_cons
   if (tid == 0) p.counters[bk] = 0u;
 }
 
+// Stages that keep two CTAs per SM (the tile ring is the bulk of the shared memory).
+template <typename T, int D, int G>
+int stages_for() {
+  using LY = FLayout<T, D, G>;
+  int s = kMaxStages;
+  while (s > 2 && LY::total(s) > (113u << 10)) --s;
+  return s;
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_t(const FullArgs& a, cudaStream_t st) {
   auto kern = full_decode_kernel<T, D, G>;
-  const size_t smem = FLayout<T, D, G>::total;
+  const int stages = stages_for<T, D, G>();
+  const size_t smem = FLayout<T, D, G>::total(stages);
   static bool attrs_set = false;  // set once, so a launch inside stream capture only launches
   if (!attrs_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -224,6 +354,7 @@ cudaError_t launch_t(const FullArgs& a, cudaStream_t st) {
   p.Hkv = a.Hkv;
   p.T = a.T;
   p.nsplit = a.nsplit;
+  p.stages = stages;
   p.scale = a.scale;
   p.q = a.q;
   p.K = a.K;
@@ -233,7 +364,7 @@ cudaError_t launch_t(const FullArgs& a, cudaStream_t st) {
   p.part = a.part;
   p.counters = a.counters;
   p.status = a.status;
-  full_decode_kernel<T, D, G><<<a.B * a.Hkv * a.nsplit, kThreads, smem, st>>>(p);
+  full_decode_kernel<T, D, G><<<a.B * a.Hkv * a.nsplit, kFThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -256,7 +387,7 @@ int full_splits(int B, int Hkv, int T) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
   const int pairs = B * Hkv;
-  int ns = (3 * sms + pairs - 1) / pairs;
+  int ns = (2 * sms + pairs - 1) / pairs;  // about two CTAs per SM over all kv-heads
   ns = ns < 1 ? 1 : ns;
   const int mx = max_full_splits(T);
   return ns > mx ? mx : ns;
