@@ -4,11 +4,12 @@
 // Split-K flash decode: the tokens of each (sequence, kv-head) are cut into `nsplit` contiguous
 // ranges, one CTA each, about two CTAs per SM. A producer warp streams the range in 32-token
 // tiles of K and V (bulk copies into a ring of shared-memory stages with a "full" and an "empty"
-// mbarrier each); eight consumer warps each take 4 rows of every tile (2 rows at a time for 8
-// query heads per kv-head) and keep their own online softmax per query head, so no CTA barrier
-// is needed until the end: logits of the rows against the G query heads of the kv-head (each lane
-// holds D / 32 channels of a row; one transpose-reduce gives every lane one (row, head) logit),
-// the running max and sum, and P.V into per-lane accumulators. The 8 warps' partials merge in
+// mbarrier each); eight consumer warps in two groups of four take alternate tiles, each warp 8
+// rows of its group's tile (as groups of 8 rows, 4 for 8 query heads per kv-head), and keep their
+// own online softmax per query head, so no CTA barrier is needed until the end: logits of the rows
+// against the G query heads of the kv-head (each lane holds D / 32 channels of a row, paired fp32
+// arithmetic; one transpose-reduce gives every lane one (row, head) logit), the running max and
+// sum, and P.V into per-lane accumulators. The 8 warps' partials merge in
 // shared memory into the split's partial (max, sum, acc) in the workspace; the last CTA of a
 // kv-head to finish (atomic ticket, no waiting) merges the splits and resets the ticket to zero
 // for the next call.
@@ -21,6 +22,8 @@ namespace {
 
 constexpr int kTT = 32;                      // tokens per tile
 constexpr int kCons = 8;                     // consumer warps
+constexpr int kGroupW = 4;                   // consumer warps that share a tile
+constexpr int kGroups = kCons / kGroupW;     // tiles in work at once
 constexpr int kFThreads = (kCons + 1) * 32;  // + the producer warp
 constexpr int kMaxStages = 8;
 
@@ -51,6 +54,29 @@ struct FLayout {
   static size_t total(int stages) { return off_ring + stage_bytes * stages; }
 };
 
+// One lane's VEP channels of a K or V row (bf16 or fp32) in shared memory, as VEP / 2 float pairs.
+template <typename T, int VEP>
+__device__ __forceinline__ void load_pairs(const T* row, int lane, float2 (&f)[VEP / 2]) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (VEP == 4) {
+      const uint2 w = reinterpret_cast<const uint2*>(row)[lane];
+      f[0] = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+      f[1] = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+    } else {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
+      f[0] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+  } else {
+    if constexpr (VEP == 4) {
+      const float4 w = reinterpret_cast<const float4*>(row)[lane];
+      f[0] = make_float2(w.x, w.y);
+      f[1] = make_float2(w.z, w.w);
+    } else {
+      f[0] = reinterpret_cast<const float2*>(row)[lane];
+    }
+  }
+}
+
 template <int G>
 __device__ __forceinline__ float pick_head(const float (&a)[G], int h) {
   float v = a[0];
@@ -63,10 +89,10 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_constant__ FParams p) {
   using LY = FLayout<T, D, G>;
   constexpr int VEP = D / 32;                // channels per lane
-  constexpr int GR = (G >= 8) ? 2 : 4;       // rows per group
+  constexpr int RPW = kTT / kGroupW;         // rows of a tile per consumer warp: 8
+  constexpr int GR = (32 / G < RPW) ? 32 / G : RPW;  // rows per group: 8 (4 for 8 heads)
   constexpr int NV = GR * G;                 // (row, head) logits of a group
   constexpr int LPV = 32 / NV;               // lanes per (row, head) after the reduce
-  constexpr int RPW = kTT / kCons;           // rows of a tile per consumer warp: 4
   static_assert(NV <= 32 && RPW % GR == 0, "unsupported head layout");
   extern __shared__ __align__(128) unsigned char sm[];
   float* q_s = reinterpret_cast<float*>(sm + LY::off_q);
@@ -93,7 +119,7 @@ __global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kCons);
+      mbar_init(&empty[s], kGroupW);
     }
     flag[1] = 0;
     mbar_init_fence();
@@ -132,24 +158,27 @@ __global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_
       for (int i = max(0, issued - NS); i < issued; ++i)
         mbar_wait(&full[i % NS], static_cast<uint32_t>((i / NS) & 1), nullptr);
     }
-  } else {  // ---- consumers
-    float qv[G][VEP];
+  } else {  // ---- consumers: warp w takes rows [8 (w % 4), 8 (w % 4) + 8) of the tiles i = w / 4 mod 2
+    constexpr int VP = VEP / 2;               // channel pairs per lane
+    float2 qv[G][VP];
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < VEP; ++e) qv[h][e] = q_s[h * D + lane * VEP + e];
-    float acc[G][VEP], mw[G], lw[G];
+      for (int e = 0; e < VP; ++e) qv[h][e] = make_float2(q_s[h * D + lane * VEP + 2 * e], q_s[h * D + lane * VEP + 2 * e + 1]);
+    float2 acc[G][VP];
+    float mw[G], lw[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       mw[h] = -CUDART_INF_F;
       lw[h] = 0.f;
 #pragma unroll
-      for (int e = 0; e < VEP; ++e) acc[h][e] = 0.f;
+      for (int e = 0; e < VP; ++e) acc[h][e] = make_float2(0.f, 0.f);
     }
     const int my_v = lane / LPV, my_r = my_v / G, my_h = my_v % G;
+    const int grp = warp / kGroupW, wi = warp % kGroupW;
     bool ok = true;
 #pragma unroll 1
-    for (int i = 0; i < ntiles; ++i) {
+    for (int i = grp; i < ntiles; i += kGroups) {
       const int st = i % NS;
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[st], static_cast<uint32_t>((i / NS) & 1), p.status));
       const int rows = ok ? min(kTT, t1 - t0 - i * kTT) : 0;
@@ -157,40 +186,24 @@ __global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_
       const T* vt = reinterpret_cast<const T*>(ring + LY::stage_bytes * st + LY::tile_bytes);
 #pragma unroll
       for (int g0 = 0; g0 < RPW; g0 += GR) {
-        const int r0 = warp * RPW + g0;  // the group's first row in the tile
+        const int r0 = wi * RPW + g0;  // the group's first row in the tile
         if (r0 >= rows) break;
         float v[NV];
 #pragma unroll
         for (int r = 0; r < GR; ++r) {
-          float kf[VEP];
+          float2 kf[VP];
           if (r0 + r < rows) {
-            const T* row = kt + (r0 + r) * D;
-            if constexpr (sizeof(T) == 2) {
-              if constexpr (VEP == 4) {
-                const uint2 w = reinterpret_cast<const uint2*>(row)[lane];
-                kf[0] = __uint_as_float(w.x << 16);
-                kf[1] = __uint_as_float(w.x & 0xffff0000u);
-                kf[2] = __uint_as_float(w.y << 16);
-                kf[3] = __uint_as_float(w.y & 0xffff0000u);
-              } else {
-                const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
-                kf[0] = __uint_as_float(w << 16);
-                kf[1] = __uint_as_float(w & 0xffff0000u);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < VEP; ++e) kf[e] = row[lane * VEP + e];
-            }
+            load_pairs<T, VEP>(kt + (r0 + r) * D, lane, kf);
           } else {
 #pragma unroll
-            for (int e = 0; e < VEP; ++e) kf[e] = 0.f;
+            for (int e = 0; e < VP; ++e) kf[e] = make_float2(0.f, 0.f);
           }
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            float s = 0.f;
+            float2 s2 = __fmul2_rn(qv[h][0], kf[0]);
 #pragma unroll
-            for (int e = 0; e < VEP; ++e) s = fmaf(qv[h][e], kf[e], s);
-            v[r * G + h] = s;
+            for (int e = 1; e < VP; ++e) s2 = __ffma2_rn(qv[h][e], kf[e], s2);
+            v[r * G + h] = s2.x + s2.y;
           }
         }
         TransposeReduce<NV, 16>::run(v, lane);  // lane holds (row my_r, head my_h)
@@ -213,35 +226,21 @@ __global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_
         for (int h = 0; h < G; ++h) {
           lw[h] = lw[h] * sc[h] + __shfl_sync(0xffffffffu, ps, h * LPV);
           mw[h] = mn[h];
+          const float2 s2 = make_float2(sc[h], sc[h]);
 #pragma unroll
-          for (int e = 0; e < VEP; ++e) acc[h][e] *= sc[h];
+          for (int e = 0; e < VP; ++e) acc[h][e] = __fmul2_rn(acc[h][e], s2);
         }
 #pragma unroll
         for (int r = 0; r < GR; ++r) {
           if (r0 + r < rows) {  // rows past the range carry weight 0 and are skipped
-            float vf[VEP];
-            const T* row = vt + (r0 + r) * D;
-            if constexpr (sizeof(T) == 2) {
-              if constexpr (VEP == 4) {
-                const uint2 w = reinterpret_cast<const uint2*>(row)[lane];
-                vf[0] = __uint_as_float(w.x << 16);
-                vf[1] = __uint_as_float(w.x & 0xffff0000u);
-                vf[2] = __uint_as_float(w.y << 16);
-                vf[3] = __uint_as_float(w.y & 0xffff0000u);
-              } else {
-                const uint32_t w = reinterpret_cast<const uint32_t*>(row)[lane];
-                vf[0] = __uint_as_float(w << 16);
-                vf[1] = __uint_as_float(w & 0xffff0000u);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < VEP; ++e) vf[e] = row[lane * VEP + e];
-            }
+            float2 vf[VP];
+            load_pairs<T, VEP>(vt + (r0 + r) * D, lane, vf);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               const float prh = __shfl_sync(0xffffffffu, pe, (r * G + h) * LPV);
+              const float2 p2 = make_float2(prh, prh);
 #pragma unroll
-              for (int e = 0; e < VEP; ++e) acc[h][e] = fmaf(prh, vf[e], acc[h][e]);
+              for (int e = 0; e < VP; ++e) acc[h][e] = __ffma2_rn(p2, vf[e], acc[h][e]);
             }
           }
         }
@@ -253,7 +252,8 @@ __global__ void __launch_bounds__(kFThreads, 2) full_decode_kernel(const __grid_
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < VEP; ++e) wacc[(warp * G + h) * D + lane * VEP + e] = acc[h][e];
+      for (int e = 0; e < VP; ++e)
+        *reinterpret_cast<float2*>(wacc + (warp * G + h) * D + lane * VEP + 2 * e) = acc[h][e];
     if (lane == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
