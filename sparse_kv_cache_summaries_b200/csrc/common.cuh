@@ -573,6 +573,13 @@ __device__ __forceinline__ void st_async_b64(uint32_t dst, uint64_t v, uint32_t 
                ::"r"(dst), "l"(v), "r"(bar) : "memory");
 }
 
+// 16 bytes (four 32-bit words) into a peer's shared memory; `dst` 16-byte aligned.
+__device__ __forceinline__ void st_async_v4(uint32_t dst, float4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(dst), "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)), "r"(__float_as_uint(v.z)),
+                 "r"(__float_as_uint(v.w)), "r"(bar) : "memory");
+}
+
 // Split cluster barrier (all threads of every CTA of the cluster). An early relaxed arrive and a
 // later wait cost almost nothing; after the wait every CTA of the cluster has started, so its
 // shared memory may be written remotely.
@@ -593,6 +600,23 @@ __device__ __forceinline__ uint64_t topk_code(uint32_t key, int idx) {
 }
 __device__ __forceinline__ int topk_index(uint64_t code) {
   return static_cast<int>(~static_cast<uint32_t>(code));
+}
+
+// Entries of a descending list of T codes (T a power of two, 0 pads the tail) above x > 0:
+// a binary search of log2(T) + 1 reads.
+// Each step is a predicated select (no branch: lanes of a warp search different lists in step).
+__device__ __forceinline__ int add_if_greater(int pos, uint64_t v, uint64_t x, int s) {
+  int r;
+  asm("{\n\t.reg .pred p;\n\tsetp.gt.u64 p, %1, %2;\n\tselp.s32 %0, %3, 0, p;\n\t}"
+      : "=r"(r) : "l"(v), "l"(x), "r"(s));
+  return pos + r;
+}
+template <int T>
+__device__ __forceinline__ int count_greater(const uint64_t* list, uint64_t x) {
+  int pos = 0;
+#pragma unroll
+  for (int s = T >> 1; s > 0; s >>= 1) pos = add_if_greater(pos, list[pos + s - 1], x, s);
+  return add_if_greater(pos, list[pos], x, 1);
 }
 
 __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int o) {

@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
   constexpr int LW = 32 * LS;  // entries of a warp Top-K list
   const int first_owner = (p.do_select && C > 1) ? 1 : 0;
   const int n_owners = C - first_owner;
-  const int per_o = (E + n_owners - 1) / n_owners;
+  const int per_o = ((E + n_owners - 1) / n_owners + 3) & ~3;  // a multiple of 4: 16-byte pushes
   const int wr = rank - first_owner;                    // this rank's output slice, if >= 0
   const int oe0 = wr >= 0 ? min(E, wr * per_o) : E, oe1 = wr >= 0 ? min(E, oe0 + per_o) : E;
   const int per_slot = (p.Kb + C - 1) / C;
@@ -293,16 +293,17 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
     }
     __syncthreads();
     // ---- 1b. log Zhat per head; compensation max, factors and sum per head
-    if (warp < G) {
+    if (warp < G) {  // the largest segment maximum, then the segment sums rescaled to it
       const int h = warp;
-      float m = -CUDART_INF_F, s = 0.f;
-      for (int t = lane; t < nseg; t += 32) lse_merge(m, s, zm_s[t * G + h], zs_s[t * G + h]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        lse_merge(m, s, m2, s2);
+      float m = -CUDART_INF_F;
+      for (int t = lane; t < nseg; t += 32) m = fmaxf(m, zm_s[t * G + h]);
+      m = warp_max(m);
+      float s = 0.f;
+      for (int t = lane; t < nseg; t += 32) {
+        const float mt = zm_s[t * G + h];
+        if (mt != -CUDART_INF_F) s = fmaf(zs_s[t * G + h], __expf(mt - m), s);
       }
+      s = warp_sum(s);
       if (lane == 0) logz[h] = (m == -CUDART_INF_F) ? -CUDART_INF_F : m + logf(s);
     }
     __syncthreads();
@@ -349,7 +350,22 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
           const uint64_t m2 = warp_merge_top32(sa, sc);
           best[0] = (k == 0) ? m2 : warp_merge_top32(best[0], m2);
         }
-        best[0] = warp_pairs_merge_top32(best[0], h64);  // warp 0: the rank's list
+        // the rank's list: each of the 8 warps' 256 entries finds its rank among them (the
+        // entries above it in all 8 lists, its own list giving its position; the searches are
+        // independent, with no branch between them) and the best 32 land in place
+        uint64_t* rl = h64 + kWarps * LW + kMaxCluster * LW;  // rank 0's merge scratch, free now
+        h64[warp * 32 + lane] = best[0];
+        if (warp == 0) rl[lane] = 0ull;
+        __syncthreads();
+        {
+          const uint64_t x = best[0];
+          int rk = 0;
+#pragma unroll
+          for (int w2 = 0; w2 < kWarps; ++w2) rk += count_greater<32>(h64 + w2 * 32, x);
+          if (x != 0ull && rk < 32) rl[rk] = x;
+        }
+        __syncthreads();
+        best[0] = rl[lane];
       } else {
         // chunks of 32 go LS at a time: one list sort, then a merge into the running list
         for (int c0 = 0; c0 * 32 < span; c0 += LS) {
@@ -373,7 +389,8 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
         }
         list_pairs_merge<LS>(best, h64);  // warp 0: the rank's list
       }
-      if (p.do_attend && warp == 0) {
+      // warp 1 when every warp holds the rank's list (lists of 32), so that warp 0 pushes it at once
+      if (p.do_attend && warp == ((LS == 1) ? 1 : 0)) {
         // speculative: this rank's likeliest picks start moving from HBM to L2 while the global
         // cut runs (about 2 K_b / C of them: the global Top-K_b holds K_b / C per rank on average)
         const int m = min(32, max(1, (2 * Kb + C - 1) / C));
@@ -464,17 +481,20 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       }
       if (warp == 0) {
         if constexpr (LS == 1) {
-          const int idx = warp_sort_asc(lane < Kb ? topk_index(src[lane]) : 0x7fffffff);
-          if (lane < Kb && p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + lane] = idx;
-          if (p.do_attend) {
-            // lane r pushes rank r's slots [r per, r per + per) into its shared memory; rank r
-            // starts as soon as its bytes land, with no cluster barrier
-            for (int q = 0; q < per_slot; ++q) {
-              const int slot = lane * per_slot + q;
-              const int v = __shfl_sync(0xffffffffu, idx, slot < 32 ? slot : 0);
-              if (lane < C && slot < Kb)
-                st_async_b32(cluster_smem_addr(&selm[q], lane), static_cast<uint32_t>(v),
-                             cluster_smem_addr(&mbar[1], lane));
+          // block order: each selected block counts the selected blocks below it; slot i goes
+          // to rank i / per_slot, which starts as soon as its bytes land (no cluster barrier)
+          int* sel_i = reinterpret_cast<int*>(dst);  // the other merge buffer, free now
+          const int mine = lane < Kb ? topk_index(src[lane]) : 0x7fffffff;
+          sel_i[lane] = mine;
+          __syncwarp();
+          int pos = 0;
+          for (int j2 = 0; j2 < Kb; ++j2) pos += sel_i[j2] < mine ? 1 : 0;
+          if (lane < Kb) {
+            if (p.sel_idx) p.sel_idx[static_cast<size_t>(pr) * Kb + pos] = mine;
+            if (p.do_attend) {
+              const int r = pos / per_slot;
+              st_async_b32(cluster_smem_addr(&selm[pos - r * per_slot], r), static_cast<uint32_t>(mine),
+                           cluster_smem_addr(&mbar[1], r));
             }
           }
         } else {
@@ -557,7 +577,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       // merge a slice of the compensation partials' channels: lanes along channels (coalesced),
       // 4 segment groups summed in a fixed order
       const int E = G * D, W = (C == 1) ? 1 : C - 1, wr = (C == 1) ? 0 : rank - 1;
-      const int per = (E + W - 1) / W;
+      const int per = ((E + W - 1) / W + 3) & ~3;  // the output slices' partition
       const int e0 = wr * per, e1 = min(E, e0 + per);
       float* mrg = red;  // scratch (the attention has not started)
       const int ei = tid % 64, sg = tid / 64;
@@ -789,14 +809,21 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const __grid_con
       st_async_b64(cluster_smem_addr(rml + (rank * G + h) * 2, o), ml, cluster_smem_addr(&mbar[2], o));
     }
   }
-  for (int i = tid; i < E; i += kThreads) {
+  for (int i = 4 * tid; i < E; i += 4 * kThreads) {  // 4 channels of one head per thread
     const int h = i / D;
-    float a = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) a = fmaf(wf[w * G + h], wacc[w * E + i], a);
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = wf[w * G + h];
+      const float4 x = *reinterpret_cast<const float4*>(wacc + w * E + i);
+      a.x = fmaf(f, x.x, a.x);
+      a.y = fmaf(f, x.y, a.y);
+      a.z = fmaf(f, x.z, a.z);
+      a.w = fmaf(f, x.w, a.w);
+    }
     const int ow = i / per_o;
-    st_async_b32(cluster_smem_addr(racc + rank * per_o + (i - ow * per_o), first_owner + ow), __float_as_uint(a),
-                 cluster_smem_addr(&mbar[2], first_owner + ow));
+    st_async_v4(cluster_smem_addr(racc + rank * per_o + (i - ow * per_o), first_owner + ow), a,
+                cluster_smem_addr(&mbar[2], first_owner + ow));
   }
   cluster_arrive();  // this rank's pushes are issued (matched by the wait before exit)
 

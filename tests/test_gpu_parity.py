@@ -131,6 +131,41 @@ def test_all_equal_scores_pick_lowest_indices():
     P.check_step(run, 256, "compkv", all_pairs(wl))
 
 
+def test_selection_held_by_one_rank():
+    # every key identical: all scores tie and the Top-K_b is the K_b lowest block indices, all in
+    # the first rank's chunk, so each rank's best few cannot settle the cut and the ranks' full
+    # lists decide it
+    wl = L32.with_(needles=0, outlier_channels=0)
+    q, K, V = synth.make_batch(wl)
+    K[:] = K[:, :, :1]
+    run = P.run_step(P.upload(wl, tensors=(q, K, V)), 512, "compkv")
+    assert torch.equal(run.sel[0], torch.arange(32, dtype=torch.int32, device="cuda").expand(8, 32))
+    P.check_step(run, 512, "compkv", all_pairs(wl))
+    sep = P.run_step(P.upload(wl, tensors=(q, K, V)), 512, "compkv", fused=False)
+    assert torch.equal(run.sel, sep.sel) and torch.equal(run.out, sep.out)
+
+
+@pytest.mark.parametrize("n_recent", [6, 40])
+def test_selection_recent_window(n_recent):
+    # keys of the last n_recent blocks pulled toward the group's mean query, so that the window
+    # dominates the selection: 6 blocks fit in what the last rank sends in the one-round
+    # exchange, 40 hold more of the Top-K_b than any rank sends
+    wl = L32.with_(needles=0)
+    q, K, V = synth.make_batch(wl)
+    G = wl.group_size
+    t0 = wl.ctx_len - 16 * n_recent
+    for g in range(wl.n_kv_heads):
+        qg = q[0, g * G:(g + 1) * G].float().mean(0)
+        K[0, g, t0:] = (K[0, g, t0:].float() + 1.5 * qg).to(K.dtype)
+    run = P.run_step(P.upload(wl, tensors=(q, K, V)), 512, "compkv")
+    P.check_step(run, 512, "compkv", all_pairs(wl))
+    if n_recent == 40:
+        recent = (run.sel >= wl.n_blocks - n_recent).sum(-1)
+        assert int(recent.min()) > 8      # more than one rank's list of the selection in the window
+    sep = P.run_step(P.upload(wl, tensors=(q, K, V)), 512, "compkv", fused=False)
+    assert torch.equal(run.sel, sep.sel) and torch.equal(run.out, sep.out)
+
+
 def test_large_logits_do_not_overflow():
     wl = L32.with_(ctx_len=4096, needles=16, needle_logit=60.0)
     run = P.run_step(P.upload(wl), 512, "compkv")
