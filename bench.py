@@ -4,8 +4,9 @@
                     [--workload llama8b_128k_b512]
 
 A step is one whole decode step of one attention layer for the whole batch: compensation-aware
-score + Top-K (compkv_score_select) and sparse compensated attention (compkv_sparse_decode), with
-the block summaries prebuilt, on seeded synthetic caches (sparse_kv_cache_summaries_b200.synth).
+score, Top-K and sparse compensated attention in one call (compkv_decode_step: the streaming score
+kernel, then the select-and-attend kernel), with the block summaries prebuilt, on seeded synthetic
+caches (sparse_kv_cache_summaries_b200.synth).
 The default workload is the Llama-3.1-8B layer at 128K context with a 512-token budget.
 
 Timing: R = 4 independent caches (K, V, summaries) are resident in HBM and the steps rotate
