@@ -9,11 +9,12 @@
 //   compensation:  (m_ref, sum n e^{lbar - m_ref}, sum n e^{lbar - m_ref} nu) over the segment
 //
 // Work split (B200): the (sequence, kv-head) tiles of 32 blocks are laid end to end and cut into
-// equal contiguous ranges, one per CTA, two CTAs per SM, so every SM streams the same number of
-// bytes whatever B and Hkv are. A CTA's range crosses at most a few (sequence, kv-head) pairs; it
-// writes one partial record per pair it touches ("segment").
+// equal contiguous ranges, one per CTA, two CTAs per SM (one, with a 6-stage ring, for 8 heads of
+// d = 128), so every SM streams the same number of bytes whatever B and Hkv are. A CTA's range
+// crosses at most a few (sequence, kv-head) pairs; it writes one partial record per pair it
+// touches ("segment").
 //
-// Pipeline: a 3-stage shared-memory ring with a "full" and an "empty" mbarrier per stage. A
+// Pipeline: a 3-stage (6-stage) shared-memory ring with a "full" and an "empty" mbarrier per stage. A
 // producer warp fills the stages (bulk copies of the tile's mean keys and mean values, 4-byte
 // cp.async of its grouped variances and counts) as soon as the 8 consumer warps have released
 // them, so no consumer ever pays for issuing a copy. Each consumer warp owns 4 blocks of every
@@ -38,7 +39,12 @@ namespace compkv {
 namespace {
 
 constexpr int kTile = kStreamTile;
-constexpr int kStages = 3;
+// Ring stages and CTAs per SM of a layout: two 9-warp CTAs per SM cap a thread at 96 registers,
+// which G = 8 query heads of d = 128 exceed (their per-lane state spills); that layout runs one
+// CTA per SM with a deeper ring instead, so the SM keeps as many bytes in flight.
+__host__ __device__ constexpr bool stream_wide(int G, int D) { return G >= 8 && D >= 128; }
+__host__ __device__ constexpr int stream_stages(int G, int D) { return stream_wide(G, D) ? 6 : 3; }
+__host__ __device__ constexpr int stream_min_ctas(int G, int D) { return stream_wide(G, D) ? 1 : 2; }
 constexpr int kBlocksPerWarp = kTile / kWarps;  // 4 (kWarps consumer warps)
 constexpr int kStreamThreads = (kWarps + 1) * 32;  // the consumers and one producer warp
 constexpr int kConsumerBar = 1;                    // named barrier of the consumer warps
@@ -64,6 +70,7 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~static_cast
 struct SLay {
   size_t stage_bytes, off_mu, off_nu, off_var, off_cnt, stage0, full, rel, wsw, q, qn, refw, red, logn, total;
   __host__ __device__ void build(int D, int G, int r, int ssz) {
+    const int kStages = stream_stages(G, D);
     off_mu = 0;
     off_nu = a16(static_cast<size_t>(ssz) * kTile * D);
     off_var = a16(off_nu + static_cast<size_t>(ssz) * kTile * D);
@@ -111,7 +118,8 @@ __device__ __forceinline__ void row_pairs(const S* row, float2 (&a)[VW / 2]) {
 
 // S: storage type of the mean key and mean value (float, or __half).
 template <typename TQ, int D, int G, int R, typename S>
-__global__ void __launch_bounds__(kStreamThreads, 2) score_stream_kernel(const __grid_constant__ StreamParams p) {
+__global__ void __launch_bounds__(kStreamThreads, stream_min_ctas(G, D)) score_stream_kernel(const __grid_constant__ StreamParams p) {
+  constexpr int kStages = stream_stages(G, D);
   extern __shared__ __align__(128) unsigned char sm[];
   SLay L;
   L.build(D, G, p.r, sizeof(S));
