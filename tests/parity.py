@@ -33,7 +33,7 @@ def layer_shape(wl: synth.Workload, **kw) -> ck.LayerShape:
 
 
 @dataclasses.dataclass
-class GpuRun:
+class GpuCase:
     wl: synth.Workload
     shape: ck.LayerShape
     q: torch.Tensor          # CPU copies (the generator's tensors)
@@ -50,20 +50,20 @@ class GpuRun:
     ws: torch.Tensor | None = None
 
 
-def upload(wl: synth.Workload, ctx_lens=None, tensors=None, summary_dtype="fp32") -> GpuRun:
+def upload(wl: synth.Workload, ctx_lens=None, tensors=None, summary_dtype="fp32") -> GpuCase:
     q, K, V = tensors if tensors is not None else synth.make_batch(wl)
     shape = layer_shape(wl, summary_dtype=summary_dtype)
     cl = None if ctx_lens is None else torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
-    return GpuRun(wl, shape, q, K, V, q.cuda(), K.cuda(), V.cuda(), cl)
+    return GpuCase(wl, shape, q, K, V, q.cuda(), K.cuda(), V.cuda(), cl)
 
 
-def run_summaries(run: GpuRun) -> ck.Summaries:
+def run_summaries(run: GpuCase) -> ck.Summaries:
     run.summ = ck.empty_summaries(run.shape)
     ck.build_summaries(run.shape, run.Kd, run.Vd, run.summ, run.ctx_lens)
     return run.summ
 
 
-def run_step(run: GpuRun, budget: int, mode: str = "compkv", fused: bool = True) -> GpuRun:
+def run_step(run: GpuCase, budget: int, mode: str = "compkv", fused: bool = True) -> GpuCase:
     if run.summ is None:
         run_summaries(run)
     s = run.shape
@@ -89,7 +89,7 @@ def rel_err(a, b) -> float:
     return float(np.max(np.abs(a - b)) / den) if den > 0 else float(np.max(np.abs(a - b)))
 
 
-def check_summaries(run: GpuRun, pairs, tol=SUMM_TOL) -> dict:
+def check_summaries(run: GpuCase, pairs, tol=SUMM_TOL) -> dict:
     worst = {"mean_k": 0.0, "var_g": 0.0, "mean_v": 0.0}
     T = run.shape.ctx_len
     for b, g in pairs:
@@ -124,7 +124,7 @@ def check_selection(sel_gpu: np.ndarray, S_ref: np.ndarray, kb: int) -> int:
     return len(diff) // 2
 
 
-def check_step(run: GpuRun, budget: int, mode: str, pairs) -> dict:
+def check_step(run: GpuCase, budget: int, mode: str, pairs) -> dict:
     """Selection, scores and outputs of sampled (b, g) pairs against the oracle."""
     s = run.shape
     G = s.group_size
@@ -166,7 +166,7 @@ def check_step(run: GpuRun, budget: int, mode: str, pairs) -> dict:
     return info
 
 
-def check_dense(run: GpuRun, out: torch.Tensor, pairs) -> float:
+def check_dense(run: GpuCase, out: torch.Tensor, pairs) -> float:
     s = run.shape
     G = s.group_size
     ctx = None if run.ctx_lens is None else run.ctx_lens.cpu().numpy()
