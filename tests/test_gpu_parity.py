@@ -197,6 +197,22 @@ def test_dense_tiny_and_llama():
         P.check_dense(run, out, all_pairs(wl))
 
 
+@pytest.mark.parametrize("G,d,dtype", [(1, 128, "bf16"), (2, 128, "bf16"), (8, 128, "bf16"),
+                                       (4, 64, "bf16"), (8, 64, "bf16"), (4, 128, "fp32")])
+def test_dense_head_layouts(G, d, dtype):
+    # every head layout of both dense kernels (tensor cores for bf16, fp32 arithmetic for fp32),
+    # with a ragged tail, more tiles per split than ring stages, and a repeated call (ticket reset)
+    wl = L32.with_(n_q_heads=2 * G, n_kv_heads=2, head_dim=d, ctx_len=12288 + 21, dtype=dtype,
+                   outlier_channels=2, needles=3)
+    run = P.upload(wl)
+    out = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), device="cuda")
+    ws = ck.new_full_workspace(run.shape)
+    for _ in range(2):
+        ck.full_decode(run.shape, run.qd, run.Kd, run.Vd, out, ws)
+    torch.cuda.synchronize()
+    P.check_dense(run, out, all_pairs(wl))
+
+
 # ------------------------------------------------------------------ full-size workloads
 
 def _full(wl, pairs, budget=None, dense=False):
