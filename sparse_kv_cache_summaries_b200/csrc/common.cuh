@@ -683,25 +683,4 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// The 8 warps' descending lists (`best` in each warp) merged pairwise in 3 levels; at level s
-// warp w (w % 2s == 0) takes warp w + s's list through `lists` and a named barrier (ids 1..7)
-// shared by those two warps only. Warp 0 returns the CTA's best 32; the other warps' return
-// values are partial. No CTA-wide barrier.
-__device__ __forceinline__ uint64_t warp_pairs_merge_top32(uint64_t best, uint64_t* lists) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int id = 1;
-#pragma unroll
-  for (int s = 1; s < kWarps; s <<= 1) {
-    if ((warp & (2 * s - 1)) == s) {  // producer at this level, done afterwards
-      lists[warp * 32 + lane] = best;
-      named_bar_arrive(id + (warp - s) / (2 * s), 64);
-    } else if ((warp & (2 * s - 1)) == 0) {
-      named_bar_sync(id + warp / (2 * s), 64);
-      best = warp_merge_top32(best, lists[(warp + s) * 32 + lane]);
-    }
-    id += kWarps / (2 * s);
-  }
-  return best;
-}
-
 }  // namespace compkv

@@ -17,8 +17,9 @@
 //     memory; the global Top-K_b under this strict order always lies inside the union of the
 //     local ones, so the result is exact. For K_b <= 32, and for K_b <= 128 when a rank holds
 //     at most 1024 blocks, the lists are each rank's best 32 LS as 64-bit codes (key, then
-//     index; LS = 1, 2 or 4 entries per lane), built and merged with warp bitonic networks;
-//     otherwise radix selection. Meanwhile the other ranks merge the compensation partials of
+//     index; LS = 1, 2 or 4 entries per lane), built with warp bitonic networks, merged within
+//     the CTA by counting (lists of 32: each entry's rank among the warps' lists) or by warp
+//     bitonic merges, and at rank 0 by a tree of warp bitonic merges; otherwise radix selection. Meanwhile the other ranks merge the compensation partials of
 //     the kv-head's segments, a slice of channels each.
 //  3. Rank c attends the c-th contiguous slice of rank 0's ordered selection (balanced whatever
 //     the blocks' positions; rank 0 writes each rank's slots into its shared memory and releases
